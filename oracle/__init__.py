@@ -1,0 +1,127 @@
+"""Test infrastructure only: the fp64 CPU oracle for segment-masked attention.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never calls it and
+shares no code with it.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, OpenMP over rows);
+this module compiles it with gcc and marshals numpy arrays through ctypes.
+What it computes, with citations, is written at the top of ``attn_oracle.c``:
+exact softmax(scale * Q K^T masked by segment-id equality) V, plus the natural
+log-sum-exp of each row, with empty rows giving out = 0 and lse = -inf.
+
+Inputs are bf16 bit patterns as ``numpy.uint16`` arrays in [B,H,S,D] order and
+int32 segment ids in [B,S] order (or None for a single segment).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_attn_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile attn_oracle.c into _attn_oracle.so (gcc, -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or \
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
+               "-shared", "-fPIC", "-std=c11", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        p = ctypes.c_void_p
+        L = ctypes.c_long
+        lib.oracle_attn_fwd_f64.argtypes = [p, p, p, p, p, p, p, L, L, L, L, L,
+                                            ctypes.c_double, ctypes.c_int]
+        lib.oracle_attn_fwd_f64.restype = ctypes.c_int
+        lib.oracle_attn_rows_f64.argtypes = [p, p, p, p, p, p, L, p, p, L, L, L, L, L,
+                                             ctypes.c_double, ctypes.c_int]
+        lib.oracle_attn_rows_f64.restype = ctypes.c_int
+        lib.oracle_attn_probs_f64.argtypes = [p, p, p, p, p, L, L, L, L, L, ctypes.c_double]
+        lib.oracle_attn_probs_f64.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _check_inputs(q, k, v, seg_q, seg_kv):
+    for name, a in (("q", q), ("k", k), ("v", v)):
+        if a.dtype != np.uint16 or a.ndim != 4 or not a.flags.c_contiguous:
+            raise TypeError(f"{name} must be a C-contiguous uint16 (bf16 bits) [B,H,S,D] array")
+    B, H, S_q, D = q.shape
+    S_kv = k.shape[2]
+    if k.shape != (B, H, S_kv, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B,H,S_kv,D] with the batch, heads and D of q")
+    if (seg_q is None) != (seg_kv is None):
+        raise ValueError("seg_q and seg_kv must both be given or both be None")
+    if seg_q is not None:
+        for name, a, s in (("seg_q", seg_q, S_q), ("seg_kv", seg_kv, S_kv)):
+            if a.dtype != np.int32 or a.shape != (B, s) or not a.flags.c_contiguous:
+                raise TypeError(f"{name} must be a C-contiguous int32 [B,{s}] array")
+    return B, H, S_q, S_kv, D
+
+
+def attn_fwd(q, k, v, seg_q=None, seg_kv=None, scale=None, nthreads=0):
+    """All rows.  Returns (out float64 [B,H,S_q,D], lse float64 [B,H,S_q])."""
+    B, H, S_q, S_kv, D = _check_inputs(q, k, v, seg_q, seg_kv)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    out = np.empty((B, H, S_q, D), np.float64)
+    lse = np.empty((B, H, S_q), np.float64)
+    rc = _load().oracle_attn_fwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv),
+                                     _ptr(out), _ptr(lse), B, H, S_q, S_kv, D,
+                                     float(scale), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_f64 failed with code {rc}")
+    return out, lse
+
+
+def attn_rows(q, k, v, rows, seg_q=None, seg_kv=None, scale=None, nthreads=0):
+    """Selected rows.  rows: int64 [n,3] of (b, h, i).
+    Returns (out float64 [n,D], lse float64 [n])."""
+    B, H, S_q, S_kv, D = _check_inputs(q, k, v, seg_q, seg_kv)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    n = rows.shape[0]
+    out = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().oracle_attn_rows_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv),
+                                      _ptr(rows), n, _ptr(out), _ptr(lse),
+                                      B, H, S_q, S_kv, D, float(scale), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_rows_f64 failed with code {rc}")
+    return out, lse
+
+
+def attn_probs(q, k, seg_q=None, seg_kv=None, scale=None):
+    """Softmax weights [B,H,S_q,S_kv] (small inputs only); masked entries are 0."""
+    B, H, S_q, D = q.shape
+    S_kv = k.shape[2]
+    _check_inputs(q, k, k, seg_q, seg_kv)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    probs = np.empty((B, H, S_q, S_kv), np.float64)
+    rc = _load().oracle_attn_probs_f64(_ptr(q), _ptr(k), _ptr(seg_q), _ptr(seg_kv),
+                                       _ptr(probs), B, H, S_q, S_kv, D, float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_probs_f64 failed with code {rc}")
+    return probs

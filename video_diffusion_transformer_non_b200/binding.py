@@ -1,0 +1,132 @@
+"""ctypes binding to the vidattn C ABI (``include/vidattn.h``).
+
+Argument marshalling only: tensors become raw pointers, streams become
+``cudaStream_t`` handles.  Every step of the attention runs in the library's
+CUDA kernels.  There is no fallback: if the library is missing or the call
+fails, these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libvidattn.so"
+_HEADER = os.path.join(os.path.dirname(_PKG), "include", "vidattn.h")
+
+VIDATTN_OK = 0
+_lib = None
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, "csrc", _LIB_NAME)
+
+
+def load_library():
+    """Load libvidattn.so (built in-tree by ``build.py``); raise if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m video_diffusion_transformer_non_b200.build` "
+            "(or __graft_entry__.build()); there is no fallback implementation")
+    lib = ctypes.CDLL(path)
+    p, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.vidattn_fwd.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, f32, p]
+    lib.vidattn_fwd.restype = i32
+    lib.vidattn_fwd_host.argtypes = [p, p, p, p, p, p, p,
+                                     p, p, p, p, p, p, p,
+                                     i32, i32, i32, i32, i32, f32, p]
+    lib.vidattn_fwd_host.restype = i32
+    lib.vidattn_status_string.argtypes = [i32]
+    lib.vidattn_status_string.restype = ctypes.c_char_p
+    lib.vidattn_release.argtypes = []
+    lib.vidattn_release.restype = None
+    lib.vidattn_device_status.argtypes = [p]
+    lib.vidattn_device_status.restype = i32
+    lib.vidattn_kernels_per_call.argtypes = [p, p, i32, i32, i32, i32, i32]
+    lib.vidattn_kernels_per_call.restype = i32
+    lib.vidattn_version.argtypes = []
+    lib.vidattn_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def exported_symbols() -> list[str]:
+    """Names of the functions declared in include/vidattn.h."""
+    with open(_HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"VIDATTN_API\s+[\w\s\*]+?\b(vidattn_\w+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return load_library().vidattn_status_string(int(status)).decode()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if hasattr(x, "ctypes"):          # numpy array (host buffer)
+        return x.ctypes.data
+    raise TypeError(f"cannot take a pointer of {type(x)}")
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def vidattn_fwd(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale, stream=None) -> int:
+    """Enqueue the forward on ``stream`` (device pointers).  Returns the status."""
+    return load_library().vidattn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv), _ptr(out), _ptr(lse),
+        int(B), int(H), int(S_q), int(S_kv), int(D), float(scale), _stream(stream))
+
+
+def vidattn_fwd_host(h_q, h_k, h_v, h_seg_q, h_seg_kv, h_out, h_lse,
+                     d_q, d_k, d_v, d_seg_q, d_seg_kv, d_out, d_lse,
+                     B, H, S_q, S_kv, D, scale, stream=None) -> int:
+    """Host buffers in and out, through caller-owned device staging buffers:
+    copies in, forward, copies out, all enqueued on ``stream``."""
+    return load_library().vidattn_fwd_host(
+        _ptr(h_q), _ptr(h_k), _ptr(h_v), _ptr(h_seg_q), _ptr(h_seg_kv), _ptr(h_out), _ptr(h_lse),
+        _ptr(d_q), _ptr(d_k), _ptr(d_v), _ptr(d_seg_q), _ptr(d_seg_kv), _ptr(d_out), _ptr(d_lse),
+        int(B), int(H), int(S_q), int(S_kv), int(D), float(scale), _stream(stream))
+
+
+def device_status(stream=None) -> int:
+    """Synchronise ``stream`` and return (and clear) the kernels' error word."""
+    return load_library().vidattn_device_status(_stream(stream))
+
+
+def kernels_per_call(seg_q, seg_kv, B, H, S_q, S_kv, D) -> int:
+    return load_library().vidattn_kernels_per_call(_ptr(seg_q), _ptr(seg_kv), int(B), int(H),
+                                                   int(S_q), int(S_kv), int(D))
+
+
+def attention(q, k, v, seg_q=None, seg_kv=None, scale=None, stream=None):
+    """Allocate out/lse with torch and run ``vidattn_fwd``.
+    q: bf16 [B,H,S_q,D]; k, v: bf16 [B,H,S_kv,D]; seg_*: int32 [B,S] or None.
+    Returns (out bf16 [B,H,S_q,D], lse fp32 [B,H,S_q]); raises on error."""
+    import torch
+    B, H, S_q, D = q.shape
+    S_kv = k.shape[2]
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S_q), dtype=torch.float32, device=q.device)
+    st = vidattn_fwd(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale, stream)
+    if st != VIDATTN_OK:
+        raise RuntimeError(f"vidattn_fwd failed: {status_string(st)} ({st})")
+    return out, lse
