@@ -1,0 +1,371 @@
+"""Benchmark of the segment-masked attention forward on B200 GPUs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one vidattn_fwd call (segment classification when ids are given,
+then the attention kernel) over one batch of the chosen workload, inputs
+already resident in HBM.  Default workload: video_480p (B1 H40 D128,
+S = 32760 tokens, one segment), a >=32k-token configuration of the kind the
+>=60%-of-peak target is quoted on.  Its inputs (~1 GB per step) are larger
+than the 126 MB L2, so no flush is needed between steps.
+
+Under torchrun (N > 1) every rank runs its own replica (independent problem,
+seeded by rank): weak scaling, no collective on the data path.  Timing is on
+the device with CUDA events, bracketed by a barrier and synchronisation, and
+the max over ranks is reported.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the only place besides the cpu_baseline leg where
+this script runs the oracle).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "bf16 video-DiT attention fwd TFLOP/s and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(bf16=float(d["bf16_tflops"]), bf16_sustained=float(d["bf16_tflops_sustained"]),
+                    hbm=float(d["hbm_gbs"]), source="measured")
+    return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+def algorithmic_bytes(w) -> int:
+    """Q, K, V read once, out and lse written once, segment ids read once."""
+    b = 2 * w.B * w.H * w.D * (2 * w.S_q + 2 * w.S_kv) + 4 * w.B * w.H * w.S_q
+    if w.segments is not None:
+        b += 4 * w.B * (w.S_q + w.S_kv)
+    return b
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 11:
+                    continue
+                if self.uuid and self.uuid not in parts[1]:
+                    continue
+                rows.append(parts)
+        os.unlink(self.tmp.name)
+        if not rows:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        util = [num(r[5]) or 0 for r in rows]
+        loaded = [num(r[2]) for r, u in zip(rows, util) if u and u > 50 and num(r[2])]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, val in zip(names, r[7:11]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(loaded or sm), "sm_max_mhz": num(rows[0][3]),
+                "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max((num(r[4]) or 0) for r in rows),
+                "reasons": sorted(reasons)}
+
+
+# -------------------------------------------------------------- reference
+
+def oracle_rows_throughput(w, inputs, n_rows, seed=0):
+    """Time the fp64 oracle on n_rows random rows of the workload.
+    Returns (TFLOP/s counted over allowed pairs of those rows, seconds, threads)."""
+    import oracle
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rows = np.stack([rng.integers(0, w.B, n_rows), rng.integers(0, w.H, n_rows),
+                     rng.integers(0, w.S_q, n_rows)], 1).astype(np.int64)
+    if inputs["seg_q"] is not None:
+        sq, sk = inputs["seg_q"], inputs["seg_kv"]
+        allowed = np.array([int(np.count_nonzero(sk[b] == sq[b, i])) for b, _, i in rows])
+    else:
+        allowed = np.full(n_rows, w.S_kv)
+    threads = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    oracle.attn_rows(inputs["q"], inputs["k"], inputs["v"], rows, inputs["seg_q"],
+                     inputs["seg_kv"], w.scale, nthreads=threads)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.D * float(allowed.sum())
+    return flops / dt / 1e12, dt, threads
+
+
+def cpu_baseline(w, inputs, target_s=12.0):
+    """Oracle on a bounded sample sized to about target_s seconds of CPU work."""
+    v, dt, thr = oracle_rows_throughput(w, inputs, 64, seed=1)
+    n = int(max(64, min(200000, 64 * target_s / max(dt, 1e-3))))
+    v, dt, thr = oracle_rows_throughput(w, inputs, n, seed=2)
+    return {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"{n} random (b,h,i) rows of {w.name} (all their allowed keys), "
+                      f"fp64 oracle, {dt:.1f} s on {thr} threads"}
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return 0
+    from video_diffusion_transformer_non_b200 import workloads as wl
+    inputs = wl.make_inputs(w)
+    v, dt, thr = oracle_rows_throughput(w, inputs, 64, seed=1)
+    # each step: a bounded sample, sized so warmup+steps take about 2 minutes
+    per_step_s = 120.0 / max(1, args.steps + args.warmup)
+    n = int(max(16, 64 * per_step_s / max(dt, 1e-3)))
+    times, vals = [], []
+    for s in range(args.warmup + args.steps):
+        v, dt, thr = oracle_rows_throughput(w, inputs, n, seed=100 + s)
+        if s >= args.warmup:
+            times.append(dt)
+            vals.append(v)
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": f"each step {n} random rows of {w.name}, fp64 oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "S_q": w.S_q, "S_kv": w.S_kv, "D": w.D,
+            "segments": None if w.segments is None else [list(r) for r in w.segments],
+            "description": w.description,
+            "l2": "inputs larger than L2 (no flush)" if algorithmic_bytes(w) > 126e6
+                  else "L2 flushed between steps",
+            "parallelism": "replicas: one independent problem per GPU"}
+
+
+# --------------------------------------------------------------------- ours
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=150)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="video_480p")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from video_diffusion_transformer_non_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, w, rank)
+
+    import torch
+    import torch.distributed as dist
+    from video_diffusion_transformer_non_b200 import binding
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    lib = binding.load_library()
+    inputs = wl.make_inputs(w, seed_offset=rank)
+    up = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = up(inputs["q"]), up(inputs["k"]), up(inputs["v"])
+    sq = None if inputs["seg_q"] is None else torch.from_numpy(inputs["seg_q"].copy()).to(dev)
+    sk = None if inputs["seg_kv"] is None else torch.from_numpy(inputs["seg_kv"].copy()).to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.S_q), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    def step():
+        st = lib.vidattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                             None if sq is None else sq.data_ptr(),
+                             None if sk is None else sk.data_ptr(),
+                             out.data_ptr(), lse.data_ptr(), w.B, w.H, w.S_q, w.S_kv, w.D,
+                             w.scale, sh)
+        if st != 0:
+            raise RuntimeError(binding.status_string(st))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if binding.device_status() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev[0].record(stream)
+    for s in range(args.steps):
+        step()
+        ev[s + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    if binding.device_status() != 0:
+        raise RuntimeError("device error during the timed region")
+    per_step = [ev[s].elapsed_time(ev[s + 1]) for s in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    total_ms_max = max_over_ranks(total_ms)
+    flops_step = wl.flops(w)
+    value = world * flops_step * args.steps / (total_ms_max * 1e-3) / 1e12
+    ms_per_step = total_ms_max / args.steps
+
+    # end to end through the host-buffer entry point: pinned inputs copied in,
+    # forward, out and lse copied back, every step
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(a).pin_memory()
+        hq, hk, hv = (pin(inputs[n].view(np.int16)) for n in ("q", "k", "v"))
+        hsq = None if inputs["seg_q"] is None else pin(inputs["seg_q"])
+        hsk = None if inputs["seg_kv"] is None else pin(inputs["seg_kv"])
+        hout = torch.empty(out.shape, dtype=torch.int16).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        ptr = lambda t: None if t is None else t.data_ptr()
+
+        def e2e_step():
+            st = lib.vidattn_fwd_host(ptr(hq), ptr(hk), ptr(hv), ptr(hsq), ptr(hsk), ptr(hout),
+                                      ptr(hlse), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                      ptr(sq), ptr(sk), out.data_ptr(), lse.data_ptr(),
+                                      w.B, w.H, w.S_q, w.S_kv, w.D, w.scale, sh)
+            if st != 0:
+                raise RuntimeError(binding.status_string(st))
+
+        n_e2e = max(3, min(args.steps, 10))
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsq, hsk) if t is not None)
+        d2h = hout.numel() * 2 + hlse.numel() * 4
+        e2e = {"value": world * flops_step * n_e2e / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
+
+    peaks = load_peaks()
+    kernel_ms = statistics.mean(per_step)   # one attention launch (+ classify) per step
+    achieved = flops_step / (kernel_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": UNIT,
+                "frac": achieved / peaks["bf16"], "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                "frac_of_sustained": achieved / peaks["bf16_sustained"],
+                "kernel": f"vidattn_fwd_kernel<{w.D}>",
+                "algorithmic_flops_per_launch": flops_step,
+                "algorithmic_bytes_per_launch": algorithmic_bytes(w)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inputs)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+            "pct_of_bf16_peak": 100.0 * value / (world * peaks["bf16"]),
+            "ms_per_step_min": min(per_step), "ms_per_step_median": statistics.median(per_step),
+            "hbm_gbs": algorithmic_bytes(w) / (kernel_ms * 1e-3) / 1e9,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * binding.kernels_per_call(
+                sq, sk, w.B, w.H, w.S_q, w.S_kv, w.D),
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,154 @@
+/*
+ * vidattn: segment-masked, non-causal multi-head attention forward for video
+ * diffusion transformers, on NVIDIA B200 (sm_100a).
+ *
+ * The operation (vidax: A Unified JAX Framework for Video Generative Models on
+ * Accelerator Meshes, §2 "3D RoPE, 3D VAEs, and flash attention": full
+ * self-attention over multi-frame patch volumes, computed without storing the
+ * query-key matrix, after FlashAttention, its reference [2]; Appendix A,
+ * Table 4, group 2 "Sharding, Parallelism & Custom Kernels", row
+ * "HunyuanVideo-1.5: RESOURCE_EXHAUSTED at 720p": segment ids replace a dense
+ * (B,H,Sq,Sk) mask and key blocks with no valid pair are skipped):
+ *
+ *   for every b < B, h < H, i < S_q, with A_i = { j < S_kv : seg_q[b,i] == seg_kv[b,j] }
+ *   (every j when both segment pointers are NULL):
+ *     out[b,h,i,:] = sum_{j in A_i} softmax_j(scale * q[b,h,i,:] . k[b,h,j,:]) * v[b,h,j,:]
+ *     lse[b,h,i]   = ln sum_{j in A_i} exp(scale * q[b,h,i,:] . k[b,h,j,:])
+ *   and for A_i empty: out[b,h,i,:] = 0, lse[b,h,i] = -inf.
+ *
+ * Arithmetic: bf16 inputs; scores, softmax statistics and the output
+ * accumulator in fp32; the softmax weights are rounded to bf16 for the
+ * weights-times-values product; out is rounded once to bf16 (nearest even).
+ *
+ * All entry points are C ABI, thread-safe for distinct streams, and never
+ * throw.  Status codes are the vidattn_status values below.
+ */
+#ifndef VIDATTN_H
+#define VIDATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define VIDATTN_API __attribute__((visibility("default")))
+#else
+#define VIDATTN_API
+#endif
+
+/* A cudaStream_t (the CUDA runtime's stream handle); NULL = legacy default stream. */
+typedef struct CUstream_st* vidattn_stream_t;
+
+typedef enum {
+  VIDATTN_OK = 0,
+  VIDATTN_ERR_NULL = 1,            /* a required pointer is NULL */
+  VIDATTN_ERR_UNSUPPORTED_D = 2,   /* D is not 64 or 128 */
+  VIDATTN_ERR_BAD_SHAPE = 3,       /* B, H, S_q or S_kv out of range */
+  VIDATTN_ERR_MISALIGNED = 4,      /* q, k, v, out not 16-byte aligned; lse, seg not 4-byte */
+  VIDATTN_ERR_CUDA = 5,            /* a CUDA call or launch failed */
+  VIDATTN_ERR_TIMEOUT = 6,         /* a kernel wait exceeded its time limit (device_status) */
+  VIDATTN_ERR_NO_DEVICE = 7,       /* the current device is not sm_100 */
+  VIDATTN_ERR_SEG_PAIR = 8         /* exactly one of seg_q, seg_kv is NULL */
+} vidattn_status;
+
+/*
+ * vidattn_fwd — the attention forward on device buffers.
+ *
+ *   q       bf16 [B,H,S_q,D]  device, contiguous (D innermost), 16-byte aligned
+ *   k, v    bf16 [B,H,S_kv,D] device, contiguous, 16-byte aligned (may be NULL
+ *           when S_kv == 0; q, out, lse may be NULL when S_q == 0)
+ *   seg_q   int32 [B,S_q]     device, contiguous, 4-byte aligned, or NULL
+ *   seg_kv  int32 [B,S_kv]    device, or NULL; NULL exactly when seg_q is NULL
+ *           (both NULL = one segment: every query sees every key).
+ *           Ids are arbitrary int32 values; a query sees a key iff the ids are
+ *           equal (padding is simply its own id).
+ *   out     bf16 [B,H,S_q,D]  device, written; 16-byte aligned
+ *   lse     fp32 [B,H,S_q]    device, written; natural log of the sum of
+ *           exp(scale * q.k) over the allowed keys; -inf for a row with none
+ *   B, H    >= 1 and <= 65535;  S_q >= 0, S_kv >= 0;  B*H*S*D < 2^31 elements
+ *           per tensor is not required (64-bit offsets), but S_q, S_kv < 2^31.
+ *   D       64 or 128
+ *   scale   multiplier of q.k inside the softmax (usually 1/sqrt(D)); any
+ *           finite value, including 0 and negative values
+ *   stream  the work is enqueued on this stream; the call does not
+ *           synchronise.  Inputs must stay valid until the stream reaches it.
+ *
+ * Ownership: the caller owns every buffer.  When segment ids are given the
+ * library keeps a small device scratch buffer per (device, stream)
+ * (16 bytes per 128 tokens of seg_q and seg_kv), allocated on first use,
+ * grown when a larger shape arrives (growing synchronises that stream), and
+ * freed by vidattn_release().  Calls on one stream are ordered, so they never
+ * share scratch in flight.
+ *
+ * Errors: argument errors return their status before anything is enqueued;
+ * launch failures return VIDATTN_ERR_CUDA.  S_q == 0 or B*H == 0 enqueues
+ * nothing and returns VIDATTN_OK.  Kernel waits are bounded (2 s); a wait
+ * that runs out sets a device error word that vidattn_device_status() reports.
+ * While that word is set, the kernels of later calls on the device return at
+ * once without writing their outputs, until vidattn_device_status() has
+ * reported and cleared it.
+ * Results are deterministic: the same inputs give bitwise the same outputs.
+ */
+VIDATTN_API int vidattn_fwd(const void* q, const void* k, const void* v,
+                            const int32_t* seg_q, const int32_t* seg_kv,
+                            void* out, float* lse,
+                            int B, int H, int S_q, int S_kv, int D, float scale,
+                            vidattn_stream_t stream);
+
+/*
+ * vidattn_fwd_host — the same operation on HOST buffers, for callers whose
+ * data lives in host memory.  h_* are host pointers (pinned memory gives
+ * asynchronous copies; pageable memory works but the copies then block);
+ * d_* are caller-owned device staging buffers of the same shapes, with the
+ * alignment rules of vidattn_fwd.  Enqueued on `stream`, in order: one
+ * host-to-device copy per input (q, k, v, then seg_q, seg_kv when given), the
+ * forward, then device-to-host copies of out and lse.  The host outputs are
+ * valid once the stream has been synchronised.  h_seg_q/h_seg_kv and
+ * d_seg_q/d_seg_kv follow the NULL rule of vidattn_fwd.
+ */
+VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h_v,
+                                 const int32_t* h_seg_q, const int32_t* h_seg_kv,
+                                 void* h_out, float* h_lse,
+                                 void* d_q, void* d_k, void* d_v,
+                                 int32_t* d_seg_q, int32_t* d_seg_kv,
+                                 void* d_out, float* d_lse,
+                                 int B, int H, int S_q, int S_kv, int D, float scale,
+                                 vidattn_stream_t stream);
+
+/* A static, human-readable name for a status code. */
+VIDATTN_API const char* vidattn_status_string(int status);
+
+/* Synchronises `stream`, then returns VIDATTN_ERR_TIMEOUT if any kernel of
+ * this library on the current device reported a timed-out wait since the last
+ * call (and clears the report), VIDATTN_ERR_CUDA if synchronising failed, else
+ * VIDATTN_OK. */
+VIDATTN_API int vidattn_device_status(vidattn_stream_t stream);
+
+/* Number of kernels one vidattn_fwd call with these arguments launches
+ * (0 when there is nothing to compute; 2 with segment ids; 1 without).
+ * Pure host logic; no CUDA call. */
+VIDATTN_API int vidattn_kernels_per_call(const int32_t* seg_q, const int32_t* seg_kv,
+                                         int B, int H, int S_q, int S_kv, int D);
+
+/* Failure-detection self-test: enqueues a one-warp kernel that waits, with the
+ * attention kernel's own bounded wait, on an mbarrier that nothing arrives on.
+ * After timeout_us microseconds (1 .. 1e6) the wait gives up, the kernel
+ * records the timeout in the device error word and returns, so a following
+ * vidattn_device_status() reports VIDATTN_ERR_TIMEOUT.  Nothing faults or
+ * hangs; the CUDA context stays usable. */
+VIDATTN_API int vidattn_selftest_timeout(int timeout_us, vidattn_stream_t stream);
+
+/* Frees the library's scratch buffers on every device after synchronising
+ * the streams they belong to.  Safe to call at any time; later calls
+ * allocate again on demand. */
+VIDATTN_API void vidattn_release(void);
+
+/* Library version and the GPU architecture it was compiled for. */
+VIDATTN_API const char* vidattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VIDATTN_H */

@@ -1,0 +1,128 @@
+"""The C-ABI boundary, on the host: the library loads, exports every entry
+point that include/vidattn.h declares, and rejects bad arguments with their
+status before any CUDA call.  No kernel runs here (every call below fails its
+argument check first, or has nothing to compute), so these pass without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import video_diffusion_transformer_non_b200 as va
+from video_diffusion_transformer_non_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# fake, never-dereferenced device addresses (16-byte aligned unless stated)
+A = 0x10000
+OK, NULL, BAD_D, BAD_SHAPE, MISALIGNED, CUDA, TIMEOUT, NO_DEVICE, SEG_PAIR = range(9)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return binding.load_library()
+
+
+def header_names():
+    with open(os.path.join(ROOT, "include", "vidattn.h")) as f:
+        return re.findall(r"VIDATTN_API\s+[\w\s\*]+?\b(vidattn_\w+)\s*\(", f.read())
+
+
+def test_header_declares_the_entry_points():
+    names = set(header_names())
+    assert {"vidattn_fwd", "vidattn_fwd_host", "vidattn_status_string", "vidattn_device_status",
+            "vidattn_kernels_per_call", "vidattn_release", "vidattn_version",
+            "vidattn_selftest_timeout"} <= names
+    assert set(binding.exported_symbols()) == names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    cdll = ctypes.CDLL(binding.library_path())
+    for name in header_names():
+        assert hasattr(cdll, name), f"{name} declared in include/vidattn.h but not exported"
+
+
+def test_version_and_status_strings(lib):
+    assert b"sm_100a" in lib.vidattn_version()
+    for code in range(9):
+        s = binding.status_string(code)
+        assert s and s != "unknown status"
+    assert binding.status_string(1234) == "unknown status"
+
+
+def call(lib, q=A, k=A, v=A, sq=None, sk=None, out=A, lse=A, B=1, H=2, Sq=256, Skv=256, D=128,
+         scale=0.125):
+    return lib.vidattn_fwd(q, k, v, sq, sk, out, lse, B, H, Sq, Skv, D, scale, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), NULL), (dict(k=None), NULL), (dict(v=None), NULL),
+    (dict(out=None), NULL), (dict(lse=None), NULL),
+    (dict(sq=A), SEG_PAIR), (dict(sk=A), SEG_PAIR),
+    (dict(D=96), BAD_D), (dict(D=256), BAD_D), (dict(D=0), BAD_D),
+    (dict(B=0), BAD_SHAPE), (dict(H=0), BAD_SHAPE), (dict(B=70000), BAD_SHAPE),
+    (dict(Sq=-1), BAD_SHAPE), (dict(Skv=-5), BAD_SHAPE),
+    (dict(q=A + 8), MISALIGNED), (dict(k=A + 2), MISALIGNED), (dict(v=A + 4), MISALIGNED),
+    (dict(out=A + 8), MISALIGNED), (dict(lse=A + 2), MISALIGNED),
+    (dict(sq=A + 1, sk=A), MISALIGNED),
+    (dict(scale=float("inf")), BAD_SHAPE), (dict(scale=float("nan")), BAD_SHAPE),
+])
+def test_argument_errors_return_before_any_launch(lib, kw, expect):
+    assert call(lib, **kw) == expect
+
+
+def test_empty_query_is_a_no_op(lib):
+    assert call(lib, Sq=0) == OK
+    assert call(lib, Sq=0, sq=A, sk=A) == OK
+
+
+def test_host_entry_point_argument_errors(lib):
+    f = lib.vidattn_fwd_host
+    args = [A] * 7 + [A] * 7 + [1, 2, 128, 128, 128, 0.1, None]
+    a = list(args); a[0] = None
+    assert f(*a) == NULL
+    a = list(args)      # host seg set, device seg NULL
+    a[10] = None; a[11] = None
+    assert f(*a) == SEG_PAIR
+    a = list(args); a[3] = None; a[4] = None     # host seg NULL, device seg set
+    assert f(*a) == SEG_PAIR
+    a = list(args); a[18] = 80
+    assert f(*a) == BAD_D
+    a = list(args); a[7] = A + 4
+    assert f(*a) == MISALIGNED
+
+
+def test_kernels_per_call(lib):
+    assert binding.kernels_per_call(None, None, 1, 2, 512, 512, 64) == 1
+    assert binding.kernels_per_call(A, A, 2, 12, 4389, 4389, 128) == 2
+    assert binding.kernels_per_call(None, None, 1, 2, 0, 512, 64) == 0
+
+
+def test_selftest_argument_range(lib):
+    assert lib.vidattn_selftest_timeout(0, None) == BAD_SHAPE
+    assert lib.vidattn_selftest_timeout(2000000, None) == BAD_SHAPE
+
+
+def test_release_without_work_is_safe(lib):
+    lib.vidattn_release()
+    lib.vidattn_release()
+
+
+def test_product_path_does_not_touch_the_oracle():
+    """The product package never imports, loads or runs anything under
+    oracle/; the oracle is test infrastructure."""
+    pkg = os.path.dirname(va.__file__)
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"\bimport\s+oracle|from\s+oracle|attn_oracle|_attn_oracle",
+                                     text), fn
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "library_path", lambda: str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        binding.load_library()

@@ -1,0 +1,211 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small and medium cases compare every row; the full-size workloads compare a
+seeded sample of rows (rows are independent, so each sampled row is an exact
+check of that row).  Tolerances: max |dout| <= 2e-2, mean |dout| <= 2e-3,
+|dlse| <= 1e-3; rows that see no key must give out == 0 and lse == -inf
+exactly.  Every call also checks guard regions around out and lse and that no
+output element is left unwritten."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from video_diffusion_transformer_non_b200 import binding
+from video_diffusion_transformer_non_b200 import workloads as wl
+
+from _gpu_helpers import (bf16_to_f64, check_all_rows, compare, run_gpu, sample_rows,
+                          to_dev_bf16, to_dev_i32)
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------ shapes, no ids
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("B,H,S_q,S_kv", [
+    (1, 1, 1, 1), (1, 2, 128, 128), (1, 2, 127, 129), (2, 2, 129, 127),
+    (1, 3, 300, 77), (1, 2, 256, 1000), (2, 1, 513, 384), (1, 1, 640, 2053),
+])
+def test_shapes_single_segment(B, H, S_q, S_kv, D):
+    c = wl.make_random(B, H, S_q, S_kv, D, seed=S_q * 7 + S_kv + D)
+    check_all_rows(c, what=f"B{B} H{H} Sq{S_q} Skv{S_kv} D{D}")
+
+
+# ----------------------------------------------------------- segment layouts
+
+def runs_case(B, H, runs, D, seed):
+    seg = wl.segment_ids(runs, B)
+    S = seg.shape[1]
+    return wl.make_random(B, H, S, S, D, seed, seg, seg.copy())
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_video_text_pad_segments(D):
+    c = runs_case(2, 3, ((700, 0), (140, 1), (37, 2)), D, 31)
+    check_all_rows(c, what="video/text/pad")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_text_and_video_shared_id_with_pad(D):
+    c = runs_case(1, 2, ((600, 0), (26, 0), (14, 1)), D, 32)
+    check_all_rows(c, what="shared id + pad")
+
+
+def test_alternating_ids_every_tile_mixed():
+    B, H, S, D = 1, 2, 515, 128
+    seg = (np.arange(S) % 2).astype(np.int32)[None]
+    c = wl.make_random(B, H, S, S, D, 33, seg, seg.copy())
+    check_all_rows(c, what="alternating")
+
+
+def test_ids_differ_between_samples_and_random_ids():
+    B, H, S, D = 3, 2, 400, 64
+    rng = np.random.Generator(np.random.PCG64(34))
+    seg_q = np.stack([np.sort(rng.integers(0, 4, S)), rng.integers(0, 3, S),
+                      np.full(S, 7)]).astype(np.int32)
+    seg_kv = np.stack([np.sort(rng.integers(0, 4, S)), rng.integers(0, 3, S),
+                       np.where(np.arange(S) < 200, 7, 8)]).astype(np.int32)
+    c = wl.make_random(B, H, S, S, D, 34, seg_q, seg_kv)
+    check_all_rows(c, what="per-sample ids")
+
+
+def test_rows_with_no_visible_key():
+    B, H, S_q, S_kv, D = 1, 2, 300, 260, 128
+    seg_q = np.where(np.arange(S_q) < 150, 5, 9).astype(np.int32)[None]   # id 9 absent
+    seg_kv = np.full((1, S_kv), 5, np.int32)
+    c = wl.make_random(B, H, S_q, S_kv, D, 35, seg_q, seg_kv)
+    stats = check_all_rows(c, what="empty rows")
+    assert stats
+    # a whole CTA with no visible key
+    seg_q2 = np.full((1, S_q), 3, np.int32)
+    c2 = wl.make_random(B, H, S_q, S_kv, D, 36, seg_q2, seg_kv)
+    out, lse = run_gpu(c2)
+    assert bool((out.float() == 0).all()) and bool(torch.isneginf(lse).all())
+
+
+def test_large_negative_and_positive_ids():
+    B, H, S, D = 1, 1, 384, 64
+    ids = np.array([-2 ** 31, 2 ** 31 - 1, 0], np.int64)
+    seg = ids[(np.arange(S) // 128) % 3].astype(np.int32)[None]
+    c = wl.make_random(B, H, S, S, D, 37, seg, seg.copy())
+    check_all_rows(c, what="extreme ids")
+
+
+# ------------------------------------------------------------------ scales
+
+@pytest.mark.parametrize("scale", [0.0, -0.125, 0.5, 1e-3])
+def test_scales(scale):
+    c = wl.make_random(1, 2, 300, 400, 128, 38)
+    check_all_rows(c, scale=scale, what=f"scale {scale}")
+
+
+def test_peaked_softmax_with_head_scaling():
+    """q and k scaled by 2 each, v ~ N(0,1) (the extreme of the 480p
+    workload's per-head scaling): near one-hot rows."""
+    c = wl.make_random(1, 2, 512, 1024, 128, 39)
+    for n in ("q", "k"):
+        c[n] = wl.f32_to_bf16_bits(wl.bf16_bits_to_f32(c[n]) * np.float32(2.0))
+    check_all_rows(c, what="peaked")
+
+
+def test_scale_zero_with_segments_gives_segment_means():
+    c = runs_case(1, 2, ((200, 0), (100, 1), (20, 2)), 128, 40)
+    check_all_rows(c, scale=0.0, what="scale 0 + ids")
+
+
+# -------------------------------------------------------------- edge cases
+
+def test_empty_key_sequence():
+    c = wl.make_random(1, 2, 200, 0, 64, 41)
+    out, lse = run_gpu(c)
+    assert bool((out.float() == 0).all()) and bool(torch.isneginf(lse).all())
+
+
+def test_empty_query_sequence_is_a_no_op():
+    q = torch.zeros(1, 2, 0, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 2, 10, 64, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(4, dtype=torch.float32, device="cuda")
+    assert binding.vidattn_fwd(k, k, k, None, None, out, lse, 1, 2, 0, 10, 64, 0.1) == 0
+    torch.cuda.synchronize()
+
+
+def test_deterministic():
+    c = runs_case(2, 2, ((500, 0), (60, 1), (9, 2)), 128, 42)
+    o1, l1 = run_gpu(c)
+    o2, l2 = run_gpu(c)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1, l2)
+
+
+def test_host_buffer_entry_point_matches_device_entry_point():
+    c = runs_case(1, 2, ((300, 0), (50, 1), (10, 2)), 128, 43)
+    out_d, lse_d = run_gpu(c)
+    B, H, S, D = c["q"].shape
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    hq, hk, hv = (pin(c[n].view(np.int16)) for n in ("q", "k", "v"))
+    hsq, hsk = pin(c["seg_q"]), pin(c["seg_kv"])
+    hout = torch.empty((B, H, S, D), dtype=torch.int16).pin_memory()
+    hlse = torch.empty((B, H, S), dtype=torch.float32).pin_memory()
+    dq, dk, dv = (torch.empty((B, H, S, D), dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    dsq, dsk = (torch.empty((B, S), dtype=torch.int32, device="cuda") for _ in range(2))
+    dout = torch.empty((B, H, S, D), dtype=torch.bfloat16, device="cuda")
+    dlse = torch.empty((B, H, S), dtype=torch.float32, device="cuda")
+    st = binding.vidattn_fwd_host(hq, hk, hv, hsq, hsk, hout, hlse, dq, dk, dv, dsq, dsk,
+                                  dout, dlse, B, H, S, S, D, c["scale"])
+    assert st == 0
+    torch.cuda.synchronize()
+    assert torch.equal(hout, out_d.view(torch.int16).cpu())
+    assert torch.equal(hlse, lse_d.cpu())
+
+
+def test_kernel_wait_timeout_is_reported_not_hung():
+    """A kernel whose barrier never completes gives up after its time limit and
+    reports through the device error word; the context stays usable."""
+    assert binding.device_status() == 0
+    assert binding.selftest_timeout(20000) == 0
+    assert binding.device_status() == 6          # VIDATTN_ERR_TIMEOUT
+    assert binding.device_status() == 0          # cleared
+    c = wl.make_random(1, 1, 128, 128, 64, 44)
+    check_all_rows(c, what="after timeout")
+
+
+def test_streams_other_than_the_current_one():
+    c = runs_case(1, 2, ((260, 0), (40, 1)), 64, 45)
+    ref_out, ref_lse = run_gpu(c)
+    s = torch.cuda.Stream()
+    q, k, v = (to_dev_bf16(c[n]) for n in ("q", "k", "v"))
+    sq, sk = to_dev_i32(c["seg_q"]), to_dev_i32(c["seg_kv"])
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        out, lse = binding.attention(q, k, v, sq, sk, c["scale"], stream=s)
+    s.synchronize()
+    assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
+    assert torch.equal(lse, ref_lse)
+
+
+# ---------------------------------------------------- the named workloads
+
+def test_workload_tiny_all_rows():
+    w = wl.WORKLOADS["tiny"]
+    check_all_rows(wl.make_inputs(w), what=w.name)
+
+
+def test_workload_joint_small_all_rows():
+    w = wl.WORKLOADS["joint_small"]
+    check_all_rows(wl.make_inputs(w), what=w.name)
+
+
+@pytest.mark.parametrize("name", ["video_480p", "cogvideox_joint", "video_720p"])
+def test_full_size_workload_sampled_rows(name):
+    w = wl.WORKLOADS[name]
+    c = wl.make_inputs(w)
+    out, lse = run_gpu(c)
+    rows = sample_rows(w.B, w.H, w.S_q, w.segments, n_random=2048, n_heads_full=4)
+    ro, rl = oracle.attn_rows(c["q"], c["k"], c["v"], rows, c["seg_q"], c["seg_kv"], c["scale"])
+    b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+    idx = torch.from_numpy(((b * w.H + h) * w.S_q + i).astype(np.int64)).cuda()
+    og = bf16_to_f64(out.reshape(-1, w.D)[idx])
+    lg = lse.reshape(-1)[idx].double().cpu().numpy()
+    compare(og, lg, ro, rl, what=name)

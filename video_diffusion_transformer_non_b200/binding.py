@@ -49,6 +49,8 @@ def load_library():
     lib.vidattn_device_status.restype = i32
     lib.vidattn_kernels_per_call.argtypes = [p, p, i32, i32, i32, i32, i32]
     lib.vidattn_kernels_per_call.restype = i32
+    lib.vidattn_selftest_timeout.argtypes = [i32, p]
+    lib.vidattn_selftest_timeout.restype = i32
     lib.vidattn_version.argtypes = []
     lib.vidattn_version.restype = ctypes.c_char_p
     _lib = lib
@@ -108,6 +110,10 @@ def vidattn_fwd_host(h_q, h_k, h_v, h_seg_q, h_seg_kv, h_out, h_lse,
 def device_status(stream=None) -> int:
     """Synchronise ``stream`` and return (and clear) the kernels' error word."""
     return load_library().vidattn_device_status(_stream(stream))
+
+
+def selftest_timeout(timeout_us: int, stream=None) -> int:
+    return load_library().vidattn_selftest_timeout(int(timeout_us), _stream(stream))
 
 
 def kernels_per_call(seg_q, seg_kv, B, H, S_q, S_kv, D) -> int:

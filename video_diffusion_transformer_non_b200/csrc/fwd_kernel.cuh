@@ -1,0 +1,506 @@
+// Segment-masked, non-causal attention forward for sm_100a.
+//
+// Computes, per (b, h, query row i), softmax over the keys j whose segment id
+// equals the query's (all keys when no ids are given) of scale * q_i . k_j,
+// applied to v, plus the natural log-sum-exp of the allowed scaled logits.
+// The full query-key matrix is never stored: scores live only in tensor memory
+// one 128x128 tile at a time and an online softmax carries the running max and
+// sum (vidax: A Unified JAX Framework for Video Generative Models on
+// Accelerator Meshes, §2 "3D RoPE, 3D VAEs, and flash attention", which
+// dispatches such attention to flash-attention kernels, its reference [2]);
+// key tiles whose ids cannot match any query of the CTA are skipped, not
+// masked (same paper, Appendix A, Table 4, group 2, row "HunyuanVideo-1.5:
+// RESOURCE_EXHAUSTED at 720p").
+//
+// One CTA = (b, h, 256 query rows as two 128-row tiles Q0, Q1).  384 threads:
+//   warps 0-3  softmax for Q0 (TMEM lanes 0-127 = the tile's rows)
+//   warps 4-7  softmax for Q1
+//   warp  8    allocates TMEM; lane 0 issues every tcgen05.mma and commit
+//   warp  9    lane 0 issues every TMA load (Q0, Q1 once; then K_j, V_j)
+//   warps 10-11 idle
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   [0,128) S0 / P0   [128,256) S1 / P1   [256,256+D) O0   [256+D,256+2D) O1
+// P (bf16, two per column) overwrites the first 64 columns of its S tile.
+// Shared memory: Q0, Q1, then a ring of kStages K-or-V tiles; every tile is
+// [D/64][128 rows][64 columns] bf16 written by TMA with 128-byte swizzle.
+//
+// Tensor-core order (one thread, in issue order; each tile pair t):
+//   S0 = Q0 K_0^T, S1 = Q1 K_0^T, then for t = 0..n-1:
+//   O0 += P0 V_t, S0 = Q0 K_{t+1}^T, O1 += P1 V_t, S1 = Q1 K_{t+1}^T
+// so the tensor core works on one Q tile while the other's softmax runs.
+// The running max is updated lazily: O is rescaled only when a row's max
+// grows by more than 2^8 (the exponentials stay <= 256 otherwise), which
+// makes the O read-modify-write in tensor memory rare.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+
+#include "ptx.cuh"
+
+namespace vidattn {
+
+constexpr int kBM = 128;        // query rows per Q tile
+constexpr int kBN = 128;        // keys per K/V tile
+constexpr int kFwdThreads = 384;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+constexpr int kErrTimeout = 1;
+
+struct FwdParams {
+  const int32_t* seg_q;     // [B,S_q] or null
+  const int32_t* seg_kv;    // [B,S_kv] or null
+  const int4* q_sum;        // [B,n_q_tiles] {min,max,uniform,0}; null without ids
+  const int4* kv_sum;       // [B,n_kv_tiles]
+  uint16_t* out;            // bf16 [B,H,S_q,D]
+  float* lse;               // fp32 [B,H,S_q]
+  int* err;                 // device error word (bit kErrTimeout: a wait timed out)
+  int H, S_q, S_kv;
+  int n_q_tiles, n_kv_tiles;
+  float c;                  // scale * log2(e)
+};
+
+template <int D>
+struct FwdCfg {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kSub = D / 64;                 // 128-byte column blocks per row
+  static constexpr int kSubBytes = 128 * 128;         // [128 rows][64 bf16]
+  static constexpr int kTileBytes = kSub * kSubBytes; // one Q, K or V tile
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  // q_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] drain[1]
+  static constexpr int kNumBars = 2 + 2 * kStages + 7;
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;   // tmem addr, abort flag
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
+  // TMEM columns: S_i / P_i at kTmemS + 128 i, O_i at kTmemO + D i
+  static constexpr uint32_t kTmemS = 0;
+  static constexpr uint32_t kTmemO = 256;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kBN, 0, 0);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
+};
+
+// Bounded wait on an mbarrier phase.  Returns false if the CTA has aborted or
+// the wait exceeded kWaitTimeoutNs (then it sets the abort flag and the
+// device error word).  Every thread that calls it observes the phase itself.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
+                                           volatile int* abort_flag, int* err,
+                                           uint64_t timeout_ns = kWaitTimeoutNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = 0;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      // give up at once if this CTA, or any CTA of this launch, already did
+      if (*abort_flag || *reinterpret_cast<volatile int*>(err)) {
+        *abort_flag = 1;
+        return false;
+      }
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > timeout_ns) {
+        *abort_flag = 1;
+        atomicOr(err, kErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// The same, with one outcome for the whole warp (needed before the
+// warp-collective tcgen05.ld/st).
+__device__ __forceinline__ bool warp_wait_phase(uint32_t bar, uint32_t parity,
+                                                volatile int* abort_flag, int* err) {
+  const bool ok = wait_phase(bar, parity, abort_flag, err);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Key tiles visited by a CTA whose query ids span [qmin, qmax]: every tile
+// without ids; with ids, the tiles whose id range intersects [qmin, qmax].
+// Every role of the CTA walks the same sequence.
+struct KvWalk {
+  const int4* kv_sum;   // this batch's summaries, or null
+  int n_kv;
+  int qmin, qmax;
+  __device__ __forceinline__ int next(int j) const {
+    if (kv_sum == nullptr) return j;
+    for (; j < n_kv; ++j) {
+      const int4 s = __ldg(kv_sum + j);
+      if (!(s.y < qmin || s.x > qmax)) return j;
+    }
+    return n_kv;
+  }
+};
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sQ, uint32_t sK) {
+  using C = FwdCfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * C::kSubBytes + (kk % 4) * 32;
+    const uint64_t a = smem_desc_sw128(sQ + off, 16, 1024);
+    const uint64_t b = smem_desc_sw128(sK + off, 16, 1024);
+    mma_ss(d_tmem, a, b, C::kIdescQK, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t sV,
+                                         bool accumulate) {
+  using C = FwdCfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk) {
+    // V is [keys][D] with D contiguous: MN-major for the B operand (N = D).
+    // 16 keys = two 8-row swizzle atoms (SBO = 1024); D/64 column blocks
+    // are kSubBytes apart (LBO).
+    const uint64_t b = smem_desc_sw128(sV + kk * 2048, C::kSubBytes, 1024);
+    mma_ts(d_tmem, p_tmem + kk * 8, b, C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    vidattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_base + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw_base);
+
+  // A wait of an earlier CTA timed out: the results are already invalid,
+  // so later CTAs end at once instead of timing out one by one.
+  if (*reinterpret_cast<volatile int*>(p.err) != 0) return;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.z;
+  const int h = blockIdx.y;
+  const int bh = b * p.H + h;
+  const int m0 = blockIdx.x * 2 * kBM;
+
+  const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
+  auto sKV = [&](int s) { return sbase + C::kOffKV + s * C::kTileBytes; };
+  auto bar = [&](int i) { return sbase + C::kOffBar + 8 * i; };
+  auto q_full = [&](int i) { return bar(i); };
+  auto kv_full = [&](int s) { return bar(2 + s); };
+  auto kv_empty = [&](int s) { return bar(2 + C::kStages + s); };
+  auto s_full = [&](int i) { return bar(2 + 2 * C::kStages + i); };
+  auto p_full = [&](int i) { return bar(4 + 2 * C::kStages + i); };
+  auto o_full = [&](int i) { return bar(6 + 2 * C::kStages + i); };
+  const uint32_t drain_bar = bar(8 + 2 * C::kStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full(0), 1);
+    mbar_init(q_full(1), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full(i), 1);
+      mbar_init(p_full(i), 128);
+      mbar_init(o_full(i), 1);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  // Query-id range of the CTA (both Q tiles) and of each Q tile.
+  const bool has_seg = p.q_sum != nullptr;
+  const int qt0 = 2 * blockIdx.x;
+  const bool has_q1 = qt0 + 1 < p.n_q_tiles;
+  int4 qs[2] = {make_int4(0, 0, 1, 0), make_int4(0, 0, 1, 0)};
+  KvWalk walk{nullptr, p.n_kv_tiles, 0, 0};
+  if (has_seg) {
+    const int4* qsum_b = p.q_sum + static_cast<int64_t>(b) * p.n_q_tiles;
+    qs[0] = __ldg(qsum_b + qt0);
+    qs[1] = has_q1 ? __ldg(qsum_b + qt0 + 1) : qs[0];
+    walk.kv_sum = p.kv_sum + static_cast<int64_t>(b) * p.n_kv_tiles;
+    walk.qmin = min(qs[0].x, qs[1].x);
+    walk.qmax = max(qs[0].y, qs[1].y);
+  }
+  const int n_kv = p.n_kv_tiles;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA loads
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int j = walk.next(0);
+      int n = 0;   // K/V loads issued
+      bool ok = true;
+      if (j < n_kv) {
+        mbar_arrive_expect_tx(q_full(0), C::kTileBytes);
+        for (int s = 0; s < C::kSub; ++s)
+          tma_load_3d(sQ[0] + s * C::kSubBytes, &tm_q, q_full(0), s * 64, m0, bh);
+      }
+      bool first = true;
+      while (ok && j < n_kv) {
+        for (int which = 0; which < 2 && ok; ++which) {   // K_j then V_j
+          const int st = n % C::kStages;
+          ok = wait_phase(kv_empty(st), ((n / C::kStages) & 1) ^ 1, abort_flag, p.err);
+          if (!ok) break;
+          mbar_arrive_expect_tx(kv_full(st), C::kTileBytes);
+          for (int s = 0; s < C::kSub; ++s)
+            tma_load_3d(sKV(st) + s * C::kSubBytes, which ? &tm_v : &tm_k, kv_full(st), s * 64,
+                        j * kBN, bh);
+          ++n;
+          if (first) {
+            first = false;
+            mbar_arrive_expect_tx(q_full(1), C::kTileBytes);
+            for (int s = 0; s < C::kSub; ++s)
+              tma_load_3d(sQ[1] + s * C::kSubBytes, &tm_q, q_full(1), s * 64, m0 + kBM, bh);
+          }
+        }
+        j = walk.next(j + 1);
+      }
+      if (!ok) {
+        // Let the loads already in flight land before the CTA can exit.
+        for (int k = (n > C::kStages ? n - C::kStages : 0); k < n; ++k) {
+          const int st = k % C::kStages;
+          volatile int never = 0;
+          wait_phase(kv_full(st), (k / C::kStages) & 1, &never, p.err);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ------------------------------------------------------- tensor core
+    if (lane == 0) {
+      int j = walk.next(0);
+      if (j < n_kv) {
+        int n = 0;   // K/V tiles consumed
+        int t = 0;
+        bool ok = wait_phase(q_full(0), 0, abort_flag, p.err);
+        int ks = n % C::kStages;
+        ok = ok && wait_phase(kv_full(ks), (n / C::kStages) & 1, abort_flag, p.err);
+        ++n;
+        if (ok) {
+          tc_fence_after();
+          issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(ks));
+          mma_commit(s_full(0));
+          ok = wait_phase(q_full(1), 0, abort_flag, p.err);
+        }
+        if (ok) {
+          tc_fence_after();
+          issue_qk<D>(tmem + (C::kTmemS + 128), sQ[1], sKV(ks));
+          mma_commit(s_full(1));
+          mma_commit(kv_empty(ks));
+        }
+        while (ok) {
+          const int vs = n % C::kStages;
+          ok = wait_phase(kv_full(vs), (n / C::kStages) & 1, abort_flag, p.err);
+          ++n;
+          if (!ok) break;
+          const int jn = walk.next(j + 1);
+          ok = wait_phase(p_full(0), t & 1, abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv<D>(tmem + C::kTmemO, tmem + C::kTmemS, sKV(vs), t > 0);
+          mma_commit(o_full(0));
+          int ks2 = 0;
+          if (jn < n_kv) {
+            ks2 = n % C::kStages;
+            ok = wait_phase(kv_full(ks2), (n / C::kStages) & 1, abort_flag, p.err);
+            ++n;
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(ks2));
+            mma_commit(s_full(0));
+          }
+          ok = wait_phase(p_full(1), t & 1, abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv<D>(tmem + (C::kTmemO + D), tmem + (C::kTmemS + 128), sKV(vs), t > 0);
+          mma_commit(o_full(1));
+          mma_commit(kv_empty(vs));
+          if (jn >= n_kv) break;
+          issue_qk<D>(tmem + (C::kTmemS + 128), sQ[1], sKV(ks2));
+          mma_commit(s_full(1));
+          mma_commit(kv_empty(ks2));
+          j = jn;
+          ++t;
+        }
+        // Every MMA issued above has finished before TMEM is released.
+        mma_commit(drain_bar);
+        volatile int never = 0;
+        wait_phase(drain_bar, 0, &never, p.err);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int qi = warp >> 2;                       // which Q tile
+    const int r = ((warp & 3) << 5) + lane;         // row in the tile = TMEM lane
+    const int row = m0 + qi * kBM + r;
+    const bool row_valid = row < p.S_q;
+    const int32_t* seg_kv_b = has_seg ? p.seg_kv + static_cast<int64_t>(b) * p.S_kv : nullptr;
+    const int my_seg = (has_seg && row_valid) ? __ldg(p.seg_q + static_cast<int64_t>(b) * p.S_q + row) : 0;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kTmemS + 128u * qi;
+    const uint32_t tO = tmem + lane_off + C::kTmemO + uint32_t(D) * qi;
+    const int4 my_qs = qs[qi];
+    const float c = p.c;
+    const bool ragged_kv = (p.S_kv % kBN) != 0;
+
+    float m_run = -INFINITY;   // running max of scale*log2(e)*s, the offset of P
+    float l_run = 0.f;         // running sum of P (fp32, before bf16 rounding)
+    int t = 0;
+    bool ok = true;
+    for (int j = walk.next(0); j < n_kv; j = walk.next(j + 1), ++t) {
+      bool masked = ragged_kv && j == n_kv - 1;
+      if (has_seg) {
+        const int4 ks = __ldg(walk.kv_sum + j);
+        masked = masked || !(my_qs.z && ks.z && my_qs.x == ks.x);
+      }
+      const bool slow = masked || !(c > 0.f);
+      ok = warp_wait_phase(s_full(qi), t & 1, abort_flag, p.err);
+      if (!ok) break;
+      tc_fence_after();
+      float s[kBN];
+      {
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) tmem_ld32(tS + 32 * k, sr[k]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          reg_fence(sr[k]);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) s[32 * k + x] = __uint_as_float(sr[k][x]);
+        }
+      }
+
+      float tile_max;
+      if (!slow) {
+        float mx = s[0];
+#pragma unroll
+        for (int x = 1; x < kBN; ++x) mx = fmaxf(mx, s[x]);
+        tile_max = mx * c;
+      } else {
+        // scaled logits; masked keys (other segment, or past S_kv) -> -inf
+        const int j0 = j * kBN;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < kBN; ++x) {
+          bool valid = (j0 + x) < p.S_kv;
+          if (has_seg && valid) valid = __ldg(seg_kv_b + j0 + x) == my_seg;
+          s[x] = valid ? s[x] * c : -INFINITY;
+          mx = fmaxf(mx, s[x]);
+        }
+        tile_max = mx;
+      }
+      const float m_new = fmaxf(m_run, tile_max);
+      const bool rescale = (m_new - m_run) > kRescaleThreshold;   // false for -inf - -inf
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = ex2(m_run - m_new);   // 0 when m_run is -inf
+        m_run = m_new;
+      }
+      const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+      float rs = 0.f;
+      uint32_t pk[2][32];
+      if (!slow) {
+#pragma unroll
+        for (int x = 0; x < kBN; x += 2) {
+          const float e0 = ex2(fmaf(s[x], c, -msub));
+          const float e1 = ex2(fmaf(s[x + 1], c, -msub));
+          rs += e0 + e1;
+          pk[x >> 6][(x >> 1) & 31] = pack_bf16x2(e0, e1);
+        }
+      } else {
+#pragma unroll
+        for (int x = 0; x < kBN; x += 2) {
+          const float e0 = ex2(s[x] - msub);
+          const float e1 = ex2(s[x + 1] - msub);
+          rs += e0 + e1;
+          pk[x >> 6][(x >> 1) & 31] = pack_bf16x2(e0, e1);
+        }
+      }
+      tmem_st32(tS, pk[0]);
+      tmem_st32(tS + 32, pk[1]);
+      l_run = l_run * alpha + rs;
+      tmem_st_wait();
+      // Rescale this tile's O rows before the next P.V accumulates into them.
+      if (__any_sync(0xffffffffu, rescale && t > 0)) {
+        ok = warp_wait_phase(o_full(qi), (t - 1) & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int k = 0; k < D / 32; ++k) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * k, o);
+          tmem_ld_wait();
+          reg_fence(o);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+          tmem_st32(tO + 32 * k, o);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(p_full(qi));
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok) {
+      if (t > 0) {
+        ok = warp_wait_phase(o_full(qi), (t - 1) & 1, abort_flag, p.err);
+        tc_fence_after();
+      }
+      const bool empty = !(l_run > 0.f);
+      const float inv_l = empty ? 0.f : 1.f / l_run;
+      const int64_t orow = static_cast<int64_t>(bh) * p.S_q + row;
+      uint16_t* out_row = p.out + orow * D;
+#pragma unroll 1
+      for (int k = 0; k < D / 32; ++k) {
+        uint32_t o[32];
+        if (t > 0 && ok) {
+          tmem_ld32(tO + 32 * k, o);
+          tmem_ld_wait();
+          reg_fence(o);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = 0u;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          w[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv_l, __uint_as_float(o[2 * x + 1]) * inv_l);
+        if (row_valid && ok) {
+          uint4* dst = reinterpret_cast<uint4*>(out_row + 32 * k);
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+        }
+      }
+      if (row_valid && ok)
+        p.lse[orow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace vidattn

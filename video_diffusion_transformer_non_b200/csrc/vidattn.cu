@@ -1,0 +1,332 @@
+// Host side of the vidattn C ABI: argument checks, TMA descriptors, the
+// segment-summary scratch cache, and kernel launches.  The operation and the
+// argument contract are documented in include/vidattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "../../include/vidattn.h"
+#include "classify.cuh"
+#include "fwd_kernel.cuh"
+
+namespace vidattn {
+
+// Device error word: kernels OR error bits into it (see kErrTimeout).
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr const char* kVersion = "vidattn 0.1 (sm_100a: TMA + tcgen05/TMEM)";
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// bf16 [BH, S, D] as a 3-D tensor map {D, S, BH}; box {64, 128, 1}, 128-byte
+// swizzle.  Rows past S read as zeros.
+bool encode_bhsd(CUtensorMap* map, const void* ptr, int64_t BH, int64_t S, int D) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(S > 0 ? S : 1), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(D) * 2 * cuuint64_t(S > 0 ? S : 1)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                   strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  bool checked = false;
+  bool ok = false;
+  bool attrs_set = false;
+};
+std::mutex g_mu;
+std::map<int, DeviceInfo> g_devices;
+
+struct Scratch {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::map<std::pair<int, cudaStream_t>, Scratch> g_scratch;
+
+int ensure_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VIDATTN_ERR_CUDA;
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& info = g_devices[dev];
+  if (!info.checked) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return VIDATTN_ERR_CUDA;
+    info.checked = true;
+    info.ok = (major == 10 && minor == 0);
+  }
+  if (!info.ok) return VIDATTN_ERR_NO_DEVICE;
+  if (!info.attrs_set) {
+    if (cudaFuncSetAttribute(vidattn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FwdCfg<64>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(vidattn_fwd_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FwdCfg<128>::kSmemBytes) != cudaSuccess)
+      return VIDATTN_ERR_CUDA;
+    info.attrs_set = true;
+  }
+  return VIDATTN_OK;
+}
+
+// Scratch of at least `bytes` for (dev, stream).  Growing synchronises the
+// stream first, so a buffer still in use by earlier work is never freed.
+void* scratch_for(int dev, cudaStream_t stream, size_t bytes) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Scratch& s = g_scratch[{dev, stream}];
+  if (s.bytes >= bytes) return s.ptr;
+  if (s.ptr) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return nullptr;
+    cudaFree(s.ptr);
+    s.ptr = nullptr;
+    s.bytes = 0;
+  }
+  size_t want = bytes < 4096 ? 4096 : bytes;
+  if (cudaMalloc(&s.ptr, want) != cudaSuccess) {
+    s.ptr = nullptr;
+    return nullptr;
+  }
+  s.bytes = want;
+  return s.ptr;
+}
+
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+int check_args(const void* q, const void* k, const void* v, const int32_t* seg_q,
+               const int32_t* seg_kv, const void* out, const float* lse, int B, int H, int S_q,
+               int S_kv, int D) {
+  if (S_q > 0 && (!q || !out || !lse)) return VIDATTN_ERR_NULL;
+  if (S_kv > 0 && (!k || !v)) return VIDATTN_ERR_NULL;
+  if ((seg_q == nullptr) != (seg_kv == nullptr)) return VIDATTN_ERR_SEG_PAIR;
+  if (D != 64 && D != 128) return VIDATTN_ERR_UNSUPPORTED_D;
+  if (B < 1 || H < 1 || B > 65535 || H > 65535 || S_q < 0 || S_kv < 0)
+    return VIDATTN_ERR_BAD_SHAPE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(lse, 4) || (seg_q && (!aligned(seg_q, 4) || !aligned(seg_kv, 4))))
+    return VIDATTN_ERR_MISALIGNED;
+  return VIDATTN_OK;
+}
+
+template <int D>
+int launch_fwd(const void* q, const void* k, const void* v, const int32_t* seg_q,
+               const int32_t* seg_kv, const int4* q_sum, const int4* kv_sum, void* out,
+               float* lse, int B, int H, int S_q, int S_kv, float scale, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  const int64_t BH = int64_t(B) * H;
+  // With no keys the K/V maps are never read; they are encoded over q.
+  const void* kp = S_kv > 0 ? k : q;
+  const void* vp = S_kv > 0 ? v : q;
+  if (!encode_bhsd(&tq, q, BH, S_q, D) || !encode_bhsd(&tk, kp, BH, S_kv, D) ||
+      !encode_bhsd(&tv, vp, BH, S_kv, D))
+    return VIDATTN_ERR_CUDA;
+  FwdParams p{};
+  p.seg_q = seg_q;
+  p.seg_kv = seg_kv;
+  p.q_sum = q_sum;
+  p.kv_sum = kv_sum;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  int* err = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_device_error) != cudaSuccess)
+    return VIDATTN_ERR_CUDA;
+  p.err = err;
+  p.H = H;
+  p.S_q = S_q;
+  p.S_kv = S_kv;
+  p.n_q_tiles = (S_q + kBM - 1) / kBM;
+  p.n_kv_tiles = (S_kv + kBN - 1) / kBN;
+  p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  dim3 grid((S_q + 2 * kBM - 1) / (2 * kBM), H, B);
+  vidattn_fwd_kernel<D><<<grid, kFwdThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? VIDATTN_OK : VIDATTN_ERR_CUDA;
+}
+
+// One warp waits on an mbarrier that nothing ever arrives on, through the
+// attention kernel's bounded wait; it gives up after timeout_ns and reports.
+__global__ void selftest_timeout_kernel(int* err, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  wait_phase(smem_u32(&bar), 0, &abort_flag, err, timeout_ns);
+  __syncwarp();
+}
+
+}  // namespace
+}  // namespace vidattn
+
+using namespace vidattn;
+
+extern "C" {
+
+VIDATTN_API const char* vidattn_version(void) { return kVersion; }
+
+VIDATTN_API const char* vidattn_status_string(int status) {
+  switch (status) {
+    case VIDATTN_OK: return "ok";
+    case VIDATTN_ERR_NULL: return "a required pointer is NULL";
+    case VIDATTN_ERR_UNSUPPORTED_D: return "head dim D must be 64 or 128";
+    case VIDATTN_ERR_BAD_SHAPE: return "B, H, S_q or S_kv out of range";
+    case VIDATTN_ERR_MISALIGNED: return "pointer misaligned (q/k/v/out need 16 bytes, lse/seg 4)";
+    case VIDATTN_ERR_CUDA: return "CUDA error";
+    case VIDATTN_ERR_TIMEOUT: return "a kernel wait timed out";
+    case VIDATTN_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
+    case VIDATTN_ERR_SEG_PAIR: return "seg_q and seg_kv must both be NULL or both be set";
+    default: return "unknown status";
+  }
+}
+
+VIDATTN_API int vidattn_kernels_per_call(const int32_t* seg_q, const int32_t* seg_kv, int B,
+                                         int H, int S_q, int S_kv, int D) {
+  (void)seg_kv;
+  (void)S_kv;
+  (void)D;
+  if (B < 1 || H < 1 || S_q < 1) return 0;
+  return seg_q ? 2 : 1;
+}
+
+VIDATTN_API int vidattn_fwd(const void* q, const void* k, const void* v, const int32_t* seg_q,
+                            const int32_t* seg_kv, void* out, float* lse, int B, int H, int S_q,
+                            int S_kv, int D, float scale, vidattn_stream_t stream_) {
+  int st = check_args(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D);
+  if (st != VIDATTN_OK) return st;
+  if (!std::isfinite(scale)) return VIDATTN_ERR_BAD_SHAPE;
+  if (S_q == 0) return VIDATTN_OK;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int dev = 0;
+  st = ensure_device(&dev);
+  if (st != VIDATTN_OK) return st;
+
+  const int4* q_sum = nullptr;
+  const int4* kv_sum = nullptr;
+  if (seg_q) {
+    const int nq = (S_q + kSegTile - 1) / kSegTile;
+    const int nk = (S_kv + kSegTile - 1) / kSegTile;
+    const size_t bytes = sizeof(int4) * size_t(B) * (size_t(nq) + size_t(nk));
+    int4* buf = static_cast<int4*>(scratch_for(dev, stream, bytes));
+    if (!buf) return VIDATTN_ERR_CUDA;
+    q_sum = buf;
+    kv_sum = buf + size_t(B) * nq;
+    dim3 grid(nq > nk ? nq : nk, B, 2);
+    seg_tile_classify_kernel<<<grid, 128, 0, stream>>>(seg_q, seg_kv, const_cast<int4*>(q_sum),
+                                                       const_cast<int4*>(kv_sum), S_q, S_kv);
+    if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
+  }
+  if (D == 64)
+    return launch_fwd<64>(q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
+                          stream);
+  return launch_fwd<128>(q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
+                         stream);
+}
+
+VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h_v,
+                                 const int32_t* h_seg_q, const int32_t* h_seg_kv, void* h_out,
+                                 float* h_lse, void* d_q, void* d_k, void* d_v, int32_t* d_seg_q,
+                                 int32_t* d_seg_kv, void* d_out, float* d_lse, int B, int H,
+                                 int S_q, int S_kv, int D, float scale,
+                                 vidattn_stream_t stream_) {
+  if (!h_q || !h_k || !h_v || !h_out || !h_lse) return VIDATTN_ERR_NULL;
+  if ((h_seg_q == nullptr) != (h_seg_kv == nullptr) ||
+      (h_seg_q == nullptr) != (d_seg_q == nullptr) ||
+      (d_seg_q == nullptr) != (d_seg_kv == nullptr))
+    return VIDATTN_ERR_SEG_PAIR;
+  int st = check_args(d_q, d_k, d_v, d_seg_q, d_seg_kv, d_out, d_lse, B, H, S_q, S_kv, D);
+  if (st != VIDATTN_OK) return st;
+  if (!std::isfinite(scale)) return VIDATTN_ERR_BAD_SHAPE;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const size_t qb = size_t(B) * H * S_q * D * 2, kvb = size_t(B) * H * S_kv * D * 2;
+  auto h2d = [&](void* d, const void* h, size_t n) {
+    return n == 0 || cudaMemcpyAsync(d, h, n, cudaMemcpyHostToDevice, stream) == cudaSuccess;
+  };
+  auto d2h = [&](void* h, const void* d, size_t n) {
+    return n == 0 || cudaMemcpyAsync(h, d, n, cudaMemcpyDeviceToHost, stream) == cudaSuccess;
+  };
+  if (!h2d(d_q, h_q, qb) || !h2d(d_k, h_k, kvb) || !h2d(d_v, h_v, kvb)) return VIDATTN_ERR_CUDA;
+  if (h_seg_q && (!h2d(d_seg_q, h_seg_q, size_t(B) * S_q * 4) ||
+                  !h2d(d_seg_kv, h_seg_kv, size_t(B) * S_kv * 4)))
+    return VIDATTN_ERR_CUDA;
+  st = vidattn_fwd(d_q, d_k, d_v, d_seg_q, d_seg_kv, d_out, d_lse, B, H, S_q, S_kv, D, scale,
+                   stream_);
+  if (st != VIDATTN_OK) return st;
+  if (!d2h(h_out, d_out, qb) || !d2h(h_lse, d_lse, size_t(B) * H * S_q * 4))
+    return VIDATTN_ERR_CUDA;
+  return VIDATTN_OK;
+}
+
+VIDATTN_API int vidattn_device_status(vidattn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return VIDATTN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess)
+    return VIDATTN_ERR_CUDA;
+  if (v != 0) {
+    int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess)
+      return VIDATTN_ERR_CUDA;
+    return VIDATTN_ERR_TIMEOUT;
+  }
+  return VIDATTN_OK;
+}
+
+VIDATTN_API int vidattn_selftest_timeout(int timeout_us, vidattn_stream_t stream_) {
+  if (timeout_us < 1 || timeout_us > 1000000) return VIDATTN_ERR_BAD_SHAPE;
+  int dev = 0;
+  int st = ensure_device(&dev);
+  if (st != VIDATTN_OK) return st;
+  int* err = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_device_error) != cudaSuccess)
+    return VIDATTN_ERR_CUDA;
+  selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream_)>>>(
+      err, 1000ull * static_cast<unsigned long long>(timeout_us));
+  return cudaGetLastError() == cudaSuccess ? VIDATTN_OK : VIDATTN_ERR_CUDA;
+}
+
+VIDATTN_API void vidattn_release(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_scratch.empty()) return;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  for (auto& kv : g_scratch) {
+    if (kv.second.ptr) {
+      cudaSetDevice(kv.first.first);
+      cudaStreamSynchronize(kv.first.second);
+      cudaFree(kv.second.ptr);
+    }
+  }
+  g_scratch.clear();
+  cudaSetDevice(prev);
+}
+
+}  // extern "C"
