@@ -202,6 +202,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="video_480p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (smaller profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args(argv)
@@ -210,6 +212,9 @@ def main(argv=None):
 
     from video_diffusion_transformer_non_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
+    if args.heads is not None:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
