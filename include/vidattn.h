@@ -50,7 +50,8 @@ typedef enum {
   VIDATTN_ERR_CUDA = 5,            /* a CUDA call or launch failed */
   VIDATTN_ERR_TIMEOUT = 6,         /* a kernel wait exceeded its time limit (device_status) */
   VIDATTN_ERR_NO_DEVICE = 7,       /* the current device is not sm_100 */
-  VIDATTN_ERR_SEG_PAIR = 8         /* exactly one of seg_q, seg_kv is NULL */
+  VIDATTN_ERR_SEG_PAIR = 8,        /* exactly one of seg_q, seg_kv is NULL */
+  VIDATTN_ERR_SCRATCH_LIMIT = 9    /* vidattn_fwd_noalloc: shape exceeds its fixed scratch */
 } vidattn_status;
 
 /*
@@ -116,6 +117,37 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
                                  void* d_out, float* d_lse,
                                  int B, int H, int S_q, int S_kv, int D, float scale,
                                  vidattn_stream_t stream);
+
+/*
+ * vidattn_fwd_noalloc — vidattn_fwd for callers that cannot allocate device
+ * memory.  The paper has no counterpart to this entry point; it exists for
+ * callers such as serving processes that hand all device memory to their own
+ * pool at start-up and forbid allocation afterwards, or code running under a
+ * fixed device-memory budget, for whom the on-demand scratch of vidattn_fwd
+ * (a cudaMalloc on first use) is not allowed.
+ *
+ * Same arguments, layouts and results as vidattn_fwd; the caller still
+ * passes every input and output.  The library allocates nothing: the segment
+ * summaries use a fixed array in the library's device memory (512 KiB on every
+ * GPU that loads the library, held until the process exits).  Limit, when
+ * segment ids are given: B * (ceil(S_q/128) + ceil(S_kv/128)) <= 32768 (for
+ * example B=1 with S_q = S_kv up to 2,097,152 tokens); larger shapes return
+ * VIDATTN_ERR_SCRATCH_LIMIT before anything is enqueued.  Without segment ids
+ * no scratch is used at all.
+ *
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's device address once (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  Calls no cudaMalloc or cudaFree.
+ * Sharing: every call on a device uses the same array, and it keeps the last
+ * call's contents; each call rewrites all of the summaries it reads before
+ * reading them, so nothing needs clearing.  Calls whose work overlaps on the
+ * GPU (for example on two streams at once) race on the array: order them.
+ */
+VIDATTN_API int vidattn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                    const int32_t* seg_q, const int32_t* seg_kv,
+                                    void* out, float* lse,
+                                    int B, int H, int S_q, int S_kv, int D, float scale,
+                                    vidattn_stream_t stream);
 
 /* A static, human-readable name for a status code. */
 VIDATTN_API const char* vidattn_status_string(int status);

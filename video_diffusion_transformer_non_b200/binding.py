@@ -37,6 +37,8 @@ def load_library():
     p, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.vidattn_fwd.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, f32, p]
     lib.vidattn_fwd.restype = i32
+    lib.vidattn_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, f32, p]
+    lib.vidattn_fwd_noalloc.restype = i32
     lib.vidattn_fwd_host.argtypes = [p, p, p, p, p, p, p,
                                      p, p, p, p, p, p, p,
                                      i32, i32, i32, i32, i32, f32, p]
@@ -92,6 +94,15 @@ def _stream(stream):
 def vidattn_fwd(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale, stream=None) -> int:
     """Enqueue the forward on ``stream`` (device pointers).  Returns the status."""
     return load_library().vidattn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv), _ptr(out), _ptr(lse),
+        int(B), int(H), int(S_q), int(S_kv), int(D), float(scale), _stream(stream))
+
+
+def vidattn_fwd_noalloc(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale,
+                        stream=None) -> int:
+    """vidattn_fwd without any device allocation (fixed library scratch, with a
+    size limit); for callers that may not allocate.  Returns the status."""
+    return load_library().vidattn_fwd_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv), _ptr(out), _ptr(lse),
         int(B), int(H), int(S_q), int(S_kv), int(D), float(scale), _stream(stream))
 

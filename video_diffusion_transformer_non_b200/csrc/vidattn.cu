@@ -21,6 +21,16 @@ namespace vidattn {
 // Device error word: kernels OR error bits into it (see kErrTimeout).
 __device__ int g_device_error = 0;
 
+// Scratch of vidattn_fwd_noalloc: the per-tile segment summaries (one int4
+// per 128 tokens of seg_q and of seg_kv, per batch entry) live in this fixed
+// array instead of memory the library allocates.  Every GPU that loads the
+// library holds it (512 KiB) until the process exits.  Host code must not
+// pass the symbol itself to a kernel: in host code it names a host-side
+// stand-in, so its device address is looked up once per device with
+// cudaGetSymbolAddress (see noalloc_scratch below).
+constexpr size_t kNoAllocMaxTiles = 32768;
+static __device__ __align__(256) int4 g_noalloc_summaries[kNoAllocMaxTiles];
+
 namespace {
 
 constexpr const char* kVersion = "vidattn 0.1 (sm_100a: TMA + tcgen05/TMEM)";
@@ -116,6 +126,22 @@ void* scratch_for(int dev, cudaStream_t stream, size_t bytes) {
   return s.ptr;
 }
 
+// Device address of g_noalloc_summaries on `dev` (which must be current),
+// looked up on the first call for that device and remembered.
+std::map<int, int4*> g_noalloc_ptr;
+int noalloc_scratch(int dev, int4** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_noalloc_ptr.find(dev);
+  if (it == g_noalloc_ptr.end()) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_summaries) != cudaSuccess || p == nullptr)
+      return VIDATTN_ERR_CUDA;
+    it = g_noalloc_ptr.emplace(dev, static_cast<int4*>(p)).first;
+  }
+  *out = it->second;
+  return VIDATTN_OK;
+}
+
 inline bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
@@ -204,6 +230,9 @@ VIDATTN_API const char* vidattn_status_string(int status) {
     case VIDATTN_ERR_TIMEOUT: return "a kernel wait timed out";
     case VIDATTN_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
     case VIDATTN_ERR_SEG_PAIR: return "seg_q and seg_kv must both be NULL or both be set";
+    case VIDATTN_ERR_SCRATCH_LIMIT:
+      return "shape too large for vidattn_fwd_noalloc's fixed scratch: "
+             "B*(ceil(S_q/128)+ceil(S_kv/128)) must be <= 32768";
     default: return "unknown status";
   }
 }
@@ -298,6 +327,48 @@ VIDATTN_API int vidattn_device_status(vidattn_stream_t stream_) {
     return VIDATTN_ERR_TIMEOUT;
   }
   return VIDATTN_OK;
+}
+
+// The forward without any allocation: like vidattn_fwd, but the segment
+// summaries go to the fixed device array g_noalloc_summaries.  Its summaries
+// are rewritten in full by the classifier before the attention kernel reads
+// them, so nothing left there by an earlier call is ever used.  Calls on one
+// device whose work overlaps on the GPU (say, on two streams at once) race on
+// the array; each device has its own copy.
+VIDATTN_API int vidattn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                    const int32_t* seg_q, const int32_t* seg_kv, void* out,
+                                    float* lse, int B, int H, int S_q, int S_kv, int D,
+                                    float scale, vidattn_stream_t stream_) {
+  int st = check_args(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D);
+  if (st != VIDATTN_OK) return st;
+  if (!std::isfinite(scale)) return VIDATTN_ERR_BAD_SHAPE;
+  if (S_q == 0) return VIDATTN_OK;
+  const int nq = (S_q + kSegTile - 1) / kSegTile;
+  const int nk = (S_kv + kSegTile - 1) / kSegTile;
+  if (seg_q && size_t(B) * (size_t(nq) + size_t(nk)) > kNoAllocMaxTiles)
+    return VIDATTN_ERR_SCRATCH_LIMIT;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int dev = 0;
+  st = ensure_device(&dev);
+  if (st != VIDATTN_OK) return st;
+  const int4* q_sum = nullptr;
+  const int4* kv_sum = nullptr;
+  if (seg_q) {
+    int4* buf = nullptr;
+    st = noalloc_scratch(dev, &buf);
+    if (st != VIDATTN_OK) return st;
+    q_sum = buf;
+    kv_sum = buf + size_t(B) * nq;
+    dim3 grid(nq > nk ? nq : nk, B, 2);
+    seg_tile_classify_kernel<<<grid, 128, 0, stream>>>(seg_q, seg_kv, buf, buf + size_t(B) * nq,
+                                                       S_q, S_kv);
+    if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
+  }
+  if (D == 64)
+    return launch_fwd<64>(q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
+                          stream);
+  return launch_fwd<128>(q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
+                         stream);
 }
 
 VIDATTN_API int vidattn_selftest_timeout(int timeout_us, vidattn_stream_t stream_) {
