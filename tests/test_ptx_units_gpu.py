@@ -23,7 +23,37 @@ def probes():
     p = ctypes.c_void_p
     lib.probe_qk_pv.argtypes = [p, p, p, p, p, p, p, ctypes.c_int, p]
     lib.probe_qk_pv.restype = ctypes.c_int
+    lib.probe_exp2_poly.argtypes = [p, p, ctypes.c_int, p]
+    lib.probe_exp2_poly.restype = ctypes.c_int
     return lib
+
+
+def test_fma_pipe_exp2_within_its_bound(probes):
+    """The polynomial 2^x used for part of the softmax exponentials: relative
+    error <= 7.5e-5 (the fitted cubic's bound) plus fp32 rounding, over
+    x in [-125, 0]; below -125 it returns 2^-125."""
+    rng = np.random.Generator(np.random.PCG64(5))
+    x = np.concatenate([np.linspace(-125.0, 0.0, 500002), rng.uniform(-30, 0, 500000),
+                        -rng.exponential(1.0, 100000), [0.0, -0.5, -1.0, -124.5, -125.0, -1e-7]])
+    x = x.astype(np.float32)
+    if x.size % 2:
+        x = np.append(x, np.float32(-3.0))
+    xd = torch.from_numpy(x).cuda()
+    yd = torch.empty_like(xd)
+    assert probes.probe_exp2_poly(xd.data_ptr(), yd.data_ptr(), x.size,
+                                  torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    y = yd.cpu().numpy().astype(np.float64)
+    ref = np.exp2(x.astype(np.float64))
+    rel = np.abs(y / ref - 1.0)
+    assert rel.max() <= 7.5e-5 + 4e-7, rel.max()
+    # below the clamp: 2^-125 times the cubic at 0
+    lo = torch.tensor([-126.0, -200.0, -1e30, -130.0], dtype=torch.float32, device="cuda")
+    lo_y = torch.empty_like(lo)
+    assert probes.probe_exp2_poly(lo.data_ptr(), lo_y.data_ptr(), 4,
+                                  torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    assert np.allclose(lo_y.cpu().numpy(), 2.0 ** -125, rtol=1e-4, atol=0)
 
 
 @pytest.mark.parametrize("D", [64, 128])

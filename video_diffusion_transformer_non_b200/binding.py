@@ -20,7 +20,8 @@ _lib = None
 
 
 def library_path() -> str:
-    return os.path.join(_PKG, "csrc", _LIB_NAME)
+    """The in-tree libvidattn.so, or the file named by VIDATTN_LIBRARY."""
+    return os.environ.get("VIDATTN_LIBRARY") or os.path.join(_PKG, "csrc", _LIB_NAME)
 
 
 def load_library():

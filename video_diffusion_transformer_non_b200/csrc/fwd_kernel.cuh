@@ -43,8 +43,13 @@ constexpr int kBM = 128;        // query rows per Q tile
 constexpr int kBN = 128;        // keys per K/V tile
 constexpr int kFwdThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr float kStaleSumLimit = 4294967296.0f;   // 2^32: bound on a tile's sum of P
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr int kErrTimeout = 1;
+// With segment ids, each CTA lists its visited key tiles in shared memory when
+// there are at most this many key tiles (S_kv <= 262144); beyond, roles walk
+// the summaries in global memory.
+constexpr int kMaxListedTiles = 2048;
 
 struct FwdParams {
   const int32_t* seg_q;     // [B,S_q] or null
@@ -72,7 +77,9 @@ struct FwdCfg {
   // q_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] drain[1]
   static constexpr int kNumBars = 2 + 2 * kStages + 7;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;   // tmem addr, abort flag
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + alignment slack
+  static constexpr int kOffWarpCnt = kOffMisc + 16;         // 12 ints (list building)
+  static constexpr int kOffList = kOffWarpCnt + 64;         // active key tiles
+  static constexpr int kSmemBytes = kOffList + 4 * kMaxListedTiles + 1024;  // + alignment slack
   // TMEM columns: S_i / P_i at kTmemS + 128 i, O_i at kTmemO + D i
   static constexpr uint32_t kTmemS = 0;
   static constexpr uint32_t kTmemO = 256;
@@ -134,6 +141,97 @@ struct KvWalk {
   }
 };
 
+// One thread's row of a 128-column S tile from tensor memory.
+__device__ __forceinline__ void load_s_row(uint32_t taddr, float (&s)[kBN]) {
+  uint32_t sr[4][32];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) tmem_ld32(taddr + 32 * k, sr[k]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    reg_fence(sr[k]);
+#pragma unroll
+    for (int x = 0; x < 32; ++x) s[32 * k + x] = __uint_as_float(sr[k][x]);
+  }
+}
+
+// Maximum of a row: four independent three-input max chains, 16 deep.
+__device__ __forceinline__ float row_max(const float (&s)[kBN]) {
+  float a[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) a[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+  for (int x = 8; x < kBN; x += 8) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) a[k] = max3f(a[k], s[x + 2 * k], s[x + 2 * k + 1]);
+  }
+  return max3f(a[0], a[1], fmaxf(a[2], a[3]));
+}
+
+// p = 2^(c*s - m) for a row of 128 scores: per 16 keys, the first 16 - kEmu
+// on the MUFU unit (ex2), the last kEmu on the FMA pipe (exp2_poly2).  The
+// bf16-rounded p go to pk (two per word, the layout of P in tensor memory);
+// returns the fp32 sum of p (four packed partial sums).
+template <int kEmu>
+__device__ __forceinline__ float exp_tile(const float (&s)[kBN], float c, float m,
+                                          uint32_t (&pk)[2][32]) {
+  const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int x = 0; x < kBN; x += 2) {
+    const float2 arg = ffma2(make_float2(s[x], s[x + 1]), c2, nm2);
+    float2 e;
+    if ((x & 15) < 16 - kEmu) {
+      e.x = ex2(arg.x);
+      e.y = ex2(arg.y);
+    } else {
+      e = exp2_poly2(arg);
+    }
+    acc[(x >> 1) & 3] = fadd2(acc[(x >> 1) & 3], e);
+    pk[x >> 6][(x >> 1) & 31] = pack_bf16x2(e.x, e.y);
+  }
+  const float2 s01 = fadd2(acc[0], acc[1]), s23 = fadd2(acc[2], acc[3]);
+  const float2 s03 = fadd2(s01, s23);
+  return s03.x + s03.y;
+}
+
+// The key-tile walk of CTA (b, pair) and, optionally, the id summary of one
+// of its two query tiles (qi), read from the classifier's output.  Each role
+// builds its own copy, so nothing stays live across the role branches.
+__device__ __forceinline__ KvWalk make_walk(const FwdParams& p, int b, int pair, int qi = -1,
+                                            int4* q_summary = nullptr) {
+  KvWalk walk{nullptr, p.n_kv_tiles, 0, 0};
+  if (p.q_sum == nullptr) {
+    if (q_summary) *q_summary = make_int4(0, 0, 1, 0);
+    return walk;
+  }
+  const int qt0 = 2 * pair;
+  const int4* qsum_b = p.q_sum + static_cast<int64_t>(b) * p.n_q_tiles;
+  const int4 q0 = __ldg(qsum_b + qt0);
+  const int4 q1 = (qt0 + 1 < p.n_q_tiles) ? __ldg(qsum_b + qt0 + 1) : q0;
+  walk.kv_sum = p.kv_sum + static_cast<int64_t>(b) * p.n_kv_tiles;
+  walk.qmin = min(q0.x, q1.x);
+  walk.qmax = max(q0.y, q1.y);
+  if (q_summary) *q_summary = (qi == 1) ? q1 : q0;
+  return walk;
+}
+
+// The sequence of key tiles a CTA visits, as every role walks it.
+//   listed: entry t of a shared-memory list: bits 0-29 = j, bit 30 + i =
+//           "Q tile i needs the masked path on this key tile";
+//   otherwise: the global walk (with ids) or every tile (without).
+struct KvSched {
+  const int* list;
+  int n_list;
+  KvWalk walk;
+  // j of the t-th visited tile (prev_j: the (t-1)-th, -1 for t = 0); n_kv when done.
+  __device__ __forceinline__ int tile(int t, int prev_j) const {
+    if (list != nullptr) return t < n_list ? (list[t] & 0x3FFFFFFF) : walk.n_kv;
+    return walk.next(prev_j + 1);
+  }
+};
+
 template <int D>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sQ, uint32_t sK) {
   using C = FwdCfg<D>;
@@ -160,7 +258,8 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   }
 }
 
-template <int D>
+// kEmu: exponentials per 16 keys computed on the FMA pipe instead of MUFU.
+template <int D, int kEmu>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     vidattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -220,29 +319,65 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-  // Query-id range of the CTA (both Q tiles) and of each Q tile.
+
   const bool has_seg = p.q_sum != nullptr;
-  const int qt0 = 2 * blockIdx.x;
-  const bool has_q1 = qt0 + 1 < p.n_q_tiles;
-  int4 qs[2] = {make_int4(0, 0, 1, 0), make_int4(0, 0, 1, 0)};
-  KvWalk walk{nullptr, p.n_kv_tiles, 0, 0};
-  if (has_seg) {
-    const int4* qsum_b = p.q_sum + static_cast<int64_t>(b) * p.n_q_tiles;
-    qs[0] = __ldg(qsum_b + qt0);
-    qs[1] = has_q1 ? __ldg(qsum_b + qt0 + 1) : qs[0];
-    walk.kv_sum = p.kv_sum + static_cast<int64_t>(b) * p.n_kv_tiles;
-    walk.qmin = min(qs[0].x, qs[1].x);
-    walk.qmax = max(qs[0].y, qs[1].y);
-  }
   const int n_kv = p.n_kv_tiles;
 
+  // With ids: compact this CTA's visited key tiles (id ranges that meet its
+  // queries' range) into shared memory, with per-Q-tile mask bits, so no role
+  // touches global memory to find its next tile.
+  int* tile_list = reinterpret_cast<int*>(smem + C::kOffList);
+  int n_list = 0;
+  const bool listed = has_seg && n_kv <= kMaxListedTiles;
+  if (listed) {
+    int4 q0, q1;
+    const KvWalk w = make_walk(p, b, blockIdx.x, 0, &q0);
+    make_walk(p, b, blockIdx.x, 1, &q1);
+    const bool ragged = (p.S_kv % kBN) != 0;
+    int* warp_cnt = reinterpret_cast<int*>(smem + C::kOffWarpCnt);
+    for (int c0 = 0; c0 < n_kv; c0 += kFwdThreads) {
+      const int jj = c0 + threadIdx.x;
+      bool act = false;
+      int entry = 0;
+      if (jj < n_kv) {
+        const int4 ks = __ldg(w.kv_sum + jj);
+        act = !(ks.y < w.qmin || ks.x > w.qmax);
+        const bool last_ragged = ragged && jj == n_kv - 1;
+        const bool m0 = last_ragged || !(q0.z && ks.z && q0.x == ks.x);
+        const bool m1 = last_ragged || !(q1.z && ks.z && q1.x == ks.x);
+        entry = jj | (m0 ? (1 << 30) : 0) | (m1 ? int(1u << 31) : 0);
+      }
+      const unsigned ballot = __ballot_sync(0xffffffffu, act);
+      if (lane == 0) warp_cnt[warp] = __popc(ballot);
+      __syncthreads();
+      int off = n_list, total = 0;
+#pragma unroll
+      for (int w2 = 0; w2 < kFwdThreads / 32; ++w2) {
+        const int cnt = warp_cnt[w2];
+        off += (w2 < warp) ? cnt : 0;
+        total += cnt;
+      }
+      if (act) tile_list[off + __popc(ballot & ((1u << lane) - 1u))] = entry;
+      n_list += total;
+      __syncthreads();
+    }
+  }
+
+  // Register split: the launch gives 168 per thread (384 x 168 = 64512);
+  // warpgroup 2 (MMA, TMA, idle warps) drops to 96 so the two softmax
+  // warpgroups can rise to 200: 128 x 96 + 256 x 200 = 63488 <= 64512.
+  // Each warpgroup executes its setmaxnreg at the head of its own branch.
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
   if (warp == 9) {
     // ------------------------------------------------------------ TMA loads
     if (lane == 0) {
+      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, blockIdx.x)};
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int j = walk.next(0);
+      int t = 0;
+      int j = sched.tile(0, -1);
       int n = 0;   // K/V loads issued
       bool ok = true;
       if (j < n_kv) {
@@ -268,7 +403,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               tma_load_3d(sQ[1] + s * C::kSubBytes, &tm_q, q_full(1), s * 64, m0 + kBM, bh);
           }
         }
-        j = walk.next(j + 1);
+        j = sched.tile(++t, j);
       }
       if (!ok) {
         // Let the loads already in flight land before the CTA can exit.
@@ -283,7 +418,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   } else if (warp == 8) {
     // ------------------------------------------------------- tensor core
     if (lane == 0) {
-      int j = walk.next(0);
+      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, blockIdx.x)};
+      int j = sched.tile(0, -1);
       if (j < n_kv) {
         int n = 0;   // K/V tiles consumed
         int t = 0;
@@ -308,7 +444,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ok = wait_phase(kv_full(vs), (n / C::kStages) & 1, abort_flag, p.err);
           ++n;
           if (!ok) break;
-          const int jn = walk.next(j + 1);
+          const int jn = sched.tile(t + 1, j);
           ok = wait_phase(p_full(0), t & 1, abort_flag, p.err);
           if (!ok) break;
           tc_fence_after();
@@ -344,7 +480,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 8) {
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
     // ------------------------------------------------------------ softmax
     const int qi = warp >> 2;                       // which Q tile
     const int r = ((warp & 3) << 5) + lane;         // row in the tile = TMEM lane
@@ -355,7 +493,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kTmemS + 128u * qi;
     const uint32_t tO = tmem + lane_off + C::kTmemO + uint32_t(D) * qi;
-    const int4 my_qs = qs[qi];
+    int4 my_qs;
+    const KvSched sched{listed ? tile_list : nullptr, n_list,
+                        make_walk(p, b, blockIdx.x, qi, &my_qs)};
     const float c = p.c;
     const bool ragged_kv = (p.S_kv % kBN) != 0;
 
@@ -363,78 +503,90 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     float l_run = 0.f;         // running sum of P (fp32, before bf16 rounding)
     int t = 0;
     bool ok = true;
-    for (int j = walk.next(0); j < n_kv; j = walk.next(j + 1), ++t) {
-      bool masked = ragged_kv && j == n_kv - 1;
-      if (has_seg) {
-        const int4 ks = __ldg(walk.kv_sum + j);
-        masked = masked || !(my_qs.z && ks.z && my_qs.x == ks.x);
+    for (int j = sched.tile(0, -1); j < n_kv; ++t, j = sched.tile(t, j)) {
+      bool masked;
+      if (listed) {
+        masked = (tile_list[t] >> (30 + qi)) & 1;
+      } else {
+        masked = ragged_kv && j == n_kv - 1;
+        if (has_seg) {
+          const int4 ks = __ldg(sched.walk.kv_sum + j);
+          masked = masked || !(my_qs.z && ks.z && my_qs.x == ks.x);
+        }
       }
       const bool slow = masked || !(c > 0.f);
       ok = warp_wait_phase(s_full(qi), t & 1, abort_flag, p.err);
       if (!ok) break;
       tc_fence_after();
-      float s[kBN];
-      {
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) tmem_ld32(tS + 32 * k, sr[k]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          reg_fence(sr[k]);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) s[32 * k + x] = __uint_as_float(sr[k][x]);
+      // P = 2^(c*s - m_run) for this tile, rounded to bf16 into pk; rs = its
+      // row sum in fp32.  Softmax does not depend on the offset m_run, so after
+      // a row's first tile the running offset is used as it stands ("stale"
+      // path, no max).  The offset only has to keep every exponential finite:
+      // if the tile's sum exceeds 2^32 the row takes the exact path instead,
+      // which computes the tile max, moves m_run up (rescaling O and l), and
+      // redoes the exponentials.  The exact path also serves masked tiles,
+      // a row's first tile, and scale <= 0.
+      float rs = 0.f, alpha = 1.f;
+      bool rescale = false;
+      // warp-uniform choice: the stale path only if every row of the warp can take it
+      bool exact = __any_sync(0xffffffffu, slow || (m_run == -INFINITY));
+      if (!exact) {
+        float s[kBN];
+        uint32_t pk[2][32];
+        load_s_row(tS, s);
+        rs = exp_tile<kEmu>(s, c, m_run, pk);
+        exact = __any_sync(0xffffffffu, !(rs <= kStaleSumLimit));
+        if (!exact) {
+          tmem_st32(tS, pk[0]);
+          tmem_st32(tS + 32, pk[1]);
         }
       }
-
-      float tile_max;
-      if (!slow) {
-        float mx = s[0];
-#pragma unroll
-        for (int x = 1; x < kBN; ++x) mx = fmaxf(mx, s[x]);
-        tile_max = mx * c;
-      } else {
-        // scaled logits; masked keys (other segment, or past S_kv) -> -inf
+      if (exact) {
+        // Two passes over the tile, 32 columns at a time, straight from
+        // tensor memory (S is intact: no P has been written yet).
         const int j0 = j * kBN;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int x = 0; x < kBN; ++x) {
+        auto allowed = [&](int x) {
           bool valid = (j0 + x) < p.S_kv;
           if (has_seg && valid) valid = __ldg(seg_kv_b + j0 + x) == my_seg;
-          s[x] = valid ? s[x] * c : -INFINITY;
-          mx = fmaxf(mx, s[x]);
-        }
-        tile_max = mx;
-      }
-      const float m_new = fmaxf(m_run, tile_max);
-      const bool rescale = (m_new - m_run) > kRescaleThreshold;   // false for -inf - -inf
-      float alpha = 1.f;
-      if (rescale) {
-        alpha = ex2(m_run - m_new);   // 0 when m_run is -inf
-        m_run = m_new;
-      }
-      const float msub = (m_run == -INFINITY) ? 0.f : m_run;
-      float rs = 0.f;
-      uint32_t pk[2][32];
-      if (!slow) {
+          return valid;
+        };
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+          uint32_t r[32];
+          tmem_ld32(tS + 32 * k, r);
+          tmem_ld_wait();
+          reg_fence(r);
 #pragma unroll
-        for (int x = 0; x < kBN; x += 2) {
-          const float e0 = ex2(fmaf(s[x], c, -msub));
-          const float e1 = ex2(fmaf(s[x + 1], c, -msub));
-          rs += e0 + e1;
-          pk[x >> 6][(x >> 1) & 31] = pack_bf16x2(e0, e1);
+          for (int x = 0; x < 32; ++x)
+            mx = fmaxf(mx, allowed(32 * k + x) ? __uint_as_float(r[x]) * c : -INFINITY);
         }
-      } else {
+        const float m_new = fmaxf(m_run, mx);
+        rescale = (m_new - m_run) > kRescaleThreshold;   // false for -inf - -inf
+        if (rescale) {
+          alpha = ex2(m_run - m_new);   // 0 when m_run is -inf
+          m_run = m_new;
+        }
+        const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+        // P chunk k (keys 32k..32k+31) lands in columns [16k, 16k+16), which
+        // hold S columns already read: chunks are processed in order.
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+          uint32_t r[32], w[16];
+          tmem_ld32(tS + 32 * k, r);
+          tmem_ld_wait();
+          reg_fence(r);
 #pragma unroll
-        for (int x = 0; x < kBN; x += 2) {
-          const float e0 = ex2(s[x] - msub);
-          const float e1 = ex2(s[x + 1] - msub);
-          rs += e0 + e1;
-          pk[x >> 6][(x >> 1) & 31] = pack_bf16x2(e0, e1);
+          for (int x = 0; x < 32; x += 2) {
+            const float e0 = allowed(32 * k + x) ? ex2(__uint_as_float(r[x]) * c - msub) : 0.f;
+            const float e1 =
+                allowed(32 * k + x + 1) ? ex2(__uint_as_float(r[x + 1]) * c - msub) : 0.f;
+            rs += e0 + e1;
+            w[x >> 1] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tS + 16 * k, w);
         }
       }
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
       l_run = l_run * alpha + rs;
       tmem_st_wait();
       // Rescale this tile's O rows before the next P.V accumulates into them.

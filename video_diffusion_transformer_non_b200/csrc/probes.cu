@@ -118,6 +118,16 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// y[i] = exp2_poly2 of x[i] (pairs), the FMA-pipe exponential of the softmax.
+__global__ void probe_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   void* p = nullptr;
   cudaDriverEntryPointQueryResult q{};
@@ -165,5 +175,15 @@ extern "C" __attribute__((visibility("default"))) int probe_qk_pv(
     probe_qk_pv_kernel<128><<<1, 128, smem, stream>>>(tq, tk, tv, static_cast<const uint16_t*>(P),
                                                        S_out, O_out, status);
   }
+  return cudaGetLastError() == cudaSuccess ? 0 : 5;
+}
+
+// x, y: n fp32 device values (n even).
+extern "C" __attribute__((visibility("default"))) int probe_exp2_poly(const float* x, float* y,
+                                                                       int n,
+                                                                       cudaStream_t stream) {
+  if (n <= 0 || (n & 1)) return 2;
+  const int pairs = n / 2;
+  probe_exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }

@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -67,8 +68,40 @@ bool encode_bhsd(CUtensorMap* map, const void* ptr, int64_t BH, int64_t S, int D
 struct DeviceInfo {
   bool checked = false;
   bool ok = false;
-  bool attrs_set = false;
+  uint32_t attrs_set = 0;   // bit (kernel variant index) once its smem limit is raised
 };
+
+using FwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                           const FwdParams);
+// Variants of the attention kernel: head dim x exponentials per 16 keys on
+// the FMA pipe.
+constexpr int kEmuChoices[] = {0, 2, 4, 6, 8};
+constexpr int kNumEmu = 5;
+template <int D>
+FwdKernel fwd_variant(int e) {
+  switch (e) {
+    case 0: return vidattn_fwd_kernel<D, 0>;
+    case 1: return vidattn_fwd_kernel<D, 2>;
+    case 2: return vidattn_fwd_kernel<D, 4>;
+    case 3: return vidattn_fwd_kernel<D, 6>;
+    default: return vidattn_fwd_kernel<D, 8>;
+  }
+}
+// Default share of exponentials moved off the MUFU unit: at D = 128 the
+// exp2 work per key tile equals the tensor-core time, at D = 64 twice it.
+// VIDATTN_EMU (0, 2, 4, 6 or 8 per 16 keys) overrides, for experiments.
+int emu_index(int D) {
+  static const int forced = [] {
+    const char* e = getenv("VIDATTN_EMU");
+    if (!e) return -1;
+    const int v = atoi(e);
+    for (int i = 0; i < kNumEmu; ++i)
+      if (kEmuChoices[i] == v) return i;
+    return -1;
+  }();
+  if (forced >= 0) return forced;
+  return D == 128 ? 2 : 4;
+}
 std::mutex g_mu;
 std::map<int, DeviceInfo> g_devices;
 
@@ -93,14 +126,15 @@ int ensure_device(int* dev_out) {
     info.ok = (major == 10 && minor == 0);
   }
   if (!info.ok) return VIDATTN_ERR_NO_DEVICE;
-  if (!info.attrs_set) {
-    if (cudaFuncSetAttribute(vidattn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdCfg<64>::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(vidattn_fwd_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdCfg<128>::kSmemBytes) != cudaSuccess)
-      return VIDATTN_ERR_CUDA;
-    info.attrs_set = true;
+  if (info.attrs_set == 0) {
+    for (int e = 0; e < kNumEmu; ++e) {
+      if (cudaFuncSetAttribute(fwd_variant<64>(e), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<64>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fwd_variant<128>(e), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<128>::kSmemBytes) != cudaSuccess)
+        return VIDATTN_ERR_CUDA;
+    }
+    info.attrs_set = 1;
   }
   return VIDATTN_OK;
 }
@@ -191,7 +225,8 @@ int launch_fwd(const void* q, const void* k, const void* v, const int32_t* seg_q
   p.n_kv_tiles = (S_kv + kBN - 1) / kBN;
   p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   dim3 grid((S_q + 2 * kBM - 1) / (2 * kBM), H, B);
-  vidattn_fwd_kernel<D><<<grid, kFwdThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
+  FwdKernel kernel = fwd_variant<D>(emu_index(D));
+  kernel<<<grid, kFwdThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? VIDATTN_OK : VIDATTN_ERR_CUDA;
 }
 
