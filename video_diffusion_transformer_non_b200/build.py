@@ -25,6 +25,8 @@ TARGETS = [
     # unit probes of the kernel's tensor-core steps, used only by the GPU tests
     (PROBES_OUT, ["probes.cu"], ["probes.cu", "fwd_kernel.cuh", "ptx.cuh"]),
 ]
+# timeline-instrumented build of the library (-DVIDATTN_TRACE), for profiling
+TRACE_OUT = os.path.join(CSRC, "libvidattn_trace.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -61,12 +63,27 @@ def build(force: bool = False, ptxas_verbose: bool = False, extra: list[str] | N
     return OUT
 
 
+def build_trace() -> str:
+    """libvidattn_trace.so: the library with per-event clock64 stamps
+    (vidattn_trace_set); same kernels otherwise."""
+    tmp = TRACE_OUT + f".tmp{os.getpid()}"
+    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
+           "-Xcompiler", "-fPIC,-fvisibility=hidden", "-cudart", "static", "-DVIDATTN_TRACE",
+           "-I", os.path.join(ROOT, "include"), "-o", tmp, os.path.join(CSRC, "vidattn.cu")]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, TRACE_OUT)
+    return TRACE_OUT
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--trace", action="store_true", help="also build libvidattn_trace.so")
     a = ap.parse_args(argv)
     print(build(force=a.force or a.verbose_ptxas, ptxas_verbose=a.verbose_ptxas))
+    if a.trace:
+        print(build_trace())
 
 
 if __name__ == "__main__":

@@ -62,7 +62,22 @@ struct FwdParams {
   int H, S_q, S_kv;
   int n_q_tiles, n_kv_tiles;
   float c;                  // scale * log2(e)
+  unsigned long long* trace; // VIDATTN_TRACE builds only: per-event clock64 stamps
 };
+
+// Timeline instrumentation, compiled in only with -DVIDATTN_TRACE: role r
+// (0 MMA, 1/2 softmax of Q tile 0/1, 3 loader), key tile t < 64, event e < 16
+// of one CTA (the middle of the grid) get a clock64() stamp.
+#ifdef VIDATTN_TRACE
+#define VIDATTN_TR(r, t, e)                                                        \
+  do {                                                                             \
+    if (trace_cta && (t) < 64) p.trace[((r) * 64 + (t)) * 16 + (e)] = clock64();   \
+  } while (0)
+#else
+#define VIDATTN_TR(r, t, e) \
+  do {                      \
+  } while (0)
+#endif
 
 template <int D>
 struct FwdCfg {
@@ -74,15 +89,22 @@ struct FwdCfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  // q_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] drain[1]
-  static constexpr int kNumBars = 2 + 2 * kStages + 7;
+  // q_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] drain[1] s_free[2]
+  static constexpr int kNumBars = 2 + 2 * kStages + 9;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;   // tmem addr, abort flag
   static constexpr int kOffWarpCnt = kOffMisc + 16;         // 12 ints (list building)
   static constexpr int kOffList = kOffWarpCnt + 64;         // active key tiles
   static constexpr int kSmemBytes = kOffList + 4 * kMaxListedTiles + 1024;  // + alignment slack
-  // TMEM columns: S_i / P_i at kTmemS + 128 i, O_i at kTmemO + D i
+  // P in its own tensor-memory columns (D = 64, where they fit) instead of
+  // over the first half of S: the next Q K^T of a tile need not wait for
+  // the P V that reads its P.
+  static constexpr bool kSepP = (D == 64);
+  // TMEM columns: S_i at kTmemS + 128 i; P_i at kTmemP + 64 i (over S_i when
+  // !kSepP); O_i at kTmemO + D i.
   static constexpr uint32_t kTmemS = 0;
-  static constexpr uint32_t kTmemO = 256;
+  static constexpr uint32_t kTmemP = kSepP ? 256 : 0;
+  static constexpr uint32_t kPStride = kSepP ? 64 : 128;
+  static constexpr uint32_t kTmemO = kSepP ? 384 : 256;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kBN, 0, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
@@ -119,8 +141,9 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
 // The same, with one outcome for the whole warp (needed before the
 // warp-collective tcgen05.ld/st).
 __device__ __forceinline__ bool warp_wait_phase(uint32_t bar, uint32_t parity,
-                                                volatile int* abort_flag, int* err) {
-  const bool ok = wait_phase(bar, parity, abort_flag, err);
+                                                volatile int* abort_flag, int* err,
+                                                uint64_t timeout_ns = kWaitTimeoutNs) {
+  const bool ok = wait_phase(bar, parity, abort_flag, err, timeout_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -240,7 +263,7 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sQ, uint32_t 
     const uint32_t off = (kk / 4) * C::kSubBytes + (kk % 4) * 32;
     const uint64_t a = smem_desc_sw128(sQ + off, 16, 1024);
     const uint64_t b = smem_desc_sw128(sK + off, 16, 1024);
-    mma_ss(d_tmem, a, b, C::kIdescQK, kk > 0 ? 1u : 0u);
+    mma_ss_elect(d_tmem, a, b, C::kIdescQK, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -254,7 +277,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
     // 16 keys = two 8-row swizzle atoms (SBO = 1024); D/64 column blocks
     // are kSubBytes apart (LBO).
     const uint64_t b = smem_desc_sw128(sV + kk * 2048, C::kSubBytes, 1024);
-    mma_ts(d_tmem, p_tmem + kk * 8, b, C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts_elect(d_tmem, p_tmem + kk * 8, b, C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -291,6 +314,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   auto p_full = [&](int i) { return bar(4 + 2 * C::kStages + i); };
   auto o_full = [&](int i) { return bar(6 + 2 * C::kStages + i); };
   const uint32_t drain_bar = bar(8 + 2 * C::kStages);
+  auto s_free = [&](int i) { return bar(9 + 2 * C::kStages + i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -305,6 +329,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(s_full(i), 1);
       mbar_init(p_full(i), 128);
       mbar_init(o_full(i), 1);
+      mbar_init(s_free(i), 128);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -322,6 +347,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const bool has_seg = p.q_sum != nullptr;
   const int n_kv = p.n_kv_tiles;
+#ifdef VIDATTN_TRACE
+  const bool trace_cta = p.trace != nullptr && blockIdx.x == gridDim.x / 2 &&
+                         blockIdx.y == gridDim.y / 2 && blockIdx.z == 0;
+#endif
 
   // With ids: compact this CTA's visited key tiles (id ranges that meet its
   // queries' range) into shared memory, with per-Q-tile mask bits, so no role
@@ -364,43 +393,53 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 
   // Register split: the launch gives 168 per thread (384 x 168 = 64512);
-  // warpgroup 2 (MMA, TMA, idle warps) drops to 96 so the two softmax
-  // warpgroups can rise to 200: 128 x 96 + 256 x 200 = 63488 <= 64512.
-  // Each warpgroup executes its setmaxnreg at the head of its own branch.
+  // warpgroup 2 (MMA, TMA, idle warps) drops so the two softmax warpgroups
+  // can rise: D = 128: 128 x 96 + 256 x 200 = 63488; D = 64 (whose softmax
+  // keeps its S row in registers): 128 x 64 + 256 x 216 = 63488; both
+  // <= 64512.  Each warpgroup executes its setmaxnreg at the head of its
+  // own branch.
   if (warp >= 8) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
+  if constexpr (D == 128) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+  }
   if (warp == 9) {
     // ------------------------------------------------------------ TMA loads
-    if (lane == 0) {
+    {  // the whole warp runs the loop; one elected lane issues
       const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, blockIdx.x)};
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+      }
       int t = 0;
       int j = sched.tile(0, -1);
       int n = 0;   // K/V loads issued
       bool ok = true;
       if (j < n_kv) {
-        mbar_arrive_expect_tx(q_full(0), C::kTileBytes);
+        mbar_arrive_expect_tx_elect(q_full(0), C::kTileBytes);
         for (int s = 0; s < C::kSub; ++s)
-          tma_load_3d(sQ[0] + s * C::kSubBytes, &tm_q, q_full(0), s * 64, m0, bh);
+          tma_load_3d_elect(sQ[0] + s * C::kSubBytes, &tm_q, q_full(0), s * 64, m0, bh);
       }
       bool first = true;
       while (ok && j < n_kv) {
         for (int which = 0; which < 2 && ok; ++which) {   // K_j then V_j
           const int st = n % C::kStages;
-          ok = wait_phase(kv_empty(st), ((n / C::kStages) & 1) ^ 1, abort_flag, p.err);
+          VIDATTN_TR(3, n, 0);
+          ok = warp_wait_phase(kv_empty(st), ((n / C::kStages) & 1) ^ 1, abort_flag, p.err);
+          VIDATTN_TR(3, n, 1);
           if (!ok) break;
-          mbar_arrive_expect_tx(kv_full(st), C::kTileBytes);
+          mbar_arrive_expect_tx_elect(kv_full(st), C::kTileBytes);
           for (int s = 0; s < C::kSub; ++s)
-            tma_load_3d(sKV(st) + s * C::kSubBytes, which ? &tm_v : &tm_k, kv_full(st), s * 64,
+            tma_load_3d_elect(sKV(st) + s * C::kSubBytes, which ? &tm_v : &tm_k, kv_full(st), s * 64,
                         j * kBN, bh);
           ++n;
           if (first) {
             first = false;
-            mbar_arrive_expect_tx(q_full(1), C::kTileBytes);
+            mbar_arrive_expect_tx_elect(q_full(1), C::kTileBytes);
             for (int s = 0; s < C::kSub; ++s)
-              tma_load_3d(sQ[1] + s * C::kSubBytes, &tm_q, q_full(1), s * 64, m0 + kBM, bh);
+              tma_load_3d_elect(sQ[1] + s * C::kSubBytes, &tm_q, q_full(1), s * 64, m0 + kBM, bh);
           }
         }
         j = sched.tile(++t, j);
@@ -410,79 +449,163 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int k = (n > C::kStages ? n - C::kStages : 0); k < n; ++k) {
           const int st = k % C::kStages;
           volatile int never = 0;
-          wait_phase(kv_full(st), (k / C::kStages) & 1, &never, p.err);
+          warp_wait_phase(kv_full(st), (k / C::kStages) & 1, &never, p.err);
         }
       }
     }
     __syncwarp();
   } else if (warp == 8) {
     // ------------------------------------------------------- tensor core
-    if (lane == 0) {
+    if (C::kSepP) {  // the whole warp runs the loop; one elected lane issues
+      // Order per tile t: S0 = Q0 K_{t+1}^T once S0_t is read, O0 += P0 V_t,
+      // S1 = Q1 K_{t+1}^T once S1_t is read, O1 += P1 V_t.  K_t is load 2t
+      // and V_t load 2t+1 of the ring.
+      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, blockIdx.x)};
+      int j = sched.tile(0, -1);
+      if (j < n_kv) {
+        auto stage = [&](int idx) { return idx % C::kStages; };
+        auto par = [&](int idx) { return uint32_t(idx / C::kStages) & 1u; };
+        int t = 0;
+        bool ok = warp_wait_phase(q_full(0), 0, abort_flag, p.err);
+        ok = ok && warp_wait_phase(kv_full(stage(0)), par(0), abort_flag, p.err);
+        if (ok) {
+          tc_fence_after();
+          issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(stage(0)));
+          mma_commit_elect(s_full(0));
+          ok = warp_wait_phase(q_full(1), 0, abort_flag, p.err);
+        }
+        if (ok) {
+          tc_fence_after();
+          issue_qk<D>(tmem + C::kTmemS + 128, sQ[1], sKV(stage(0)));
+          mma_commit_elect(s_full(1));
+          mma_commit_elect(kv_empty(stage(0)));
+        }
+        while (ok) {
+          const int jn = sched.tile(t + 1, j);
+          const bool more = jn < n_kv;
+          const int kn = 2 * (t + 1), vi = 2 * t + 1;
+          VIDATTN_TR(0, t, 0);
+          if (more) {
+            ok = warp_wait_phase(kv_full(stage(kn)), par(kn), abort_flag, p.err) &&
+                 warp_wait_phase(s_free(0), t & 1, abort_flag, p.err);
+            VIDATTN_TR(0, t, 1);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(stage(kn)));
+            mma_commit_elect(s_full(0));
+            VIDATTN_TR(0, t, 2);
+          }
+          ok = warp_wait_phase(kv_full(stage(vi)), par(vi), abort_flag, p.err) &&
+               warp_wait_phase(p_full(0), t & 1, abort_flag, p.err);
+          VIDATTN_TR(0, t, 3);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv<D>(tmem + C::kTmemO, tmem + C::kTmemP, sKV(stage(vi)), t > 0);
+          mma_commit_elect(o_full(0));
+          VIDATTN_TR(0, t, 4);
+          if (more) {
+            ok = warp_wait_phase(s_free(1), t & 1, abort_flag, p.err);
+            VIDATTN_TR(0, t, 5);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk<D>(tmem + C::kTmemS + 128, sQ[1], sKV(stage(kn)));
+            mma_commit_elect(s_full(1));
+            mma_commit_elect(kv_empty(stage(kn)));
+            VIDATTN_TR(0, t, 6);
+          }
+          ok = warp_wait_phase(p_full(1), t & 1, abort_flag, p.err);
+          VIDATTN_TR(0, t, 7);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv<D>(tmem + C::kTmemO + D, tmem + C::kTmemP + C::kPStride, sKV(stage(vi)),
+                      t > 0);
+          mma_commit_elect(o_full(1));
+          mma_commit_elect(kv_empty(stage(vi)));
+          VIDATTN_TR(0, t, 8);
+          if (!more) break;
+          j = jn;
+          ++t;
+        }
+        mma_commit_elect(drain_bar);
+        volatile int never = 0;
+        warp_wait_phase(drain_bar, 0, &never, p.err);
+      }
+    } else {
       const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, blockIdx.x)};
       int j = sched.tile(0, -1);
       if (j < n_kv) {
         int n = 0;   // K/V tiles consumed
         int t = 0;
-        bool ok = wait_phase(q_full(0), 0, abort_flag, p.err);
+        bool ok = warp_wait_phase(q_full(0), 0, abort_flag, p.err);
         int ks = n % C::kStages;
-        ok = ok && wait_phase(kv_full(ks), (n / C::kStages) & 1, abort_flag, p.err);
+        ok = ok && warp_wait_phase(kv_full(ks), (n / C::kStages) & 1, abort_flag, p.err);
         ++n;
         if (ok) {
           tc_fence_after();
           issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(ks));
-          mma_commit(s_full(0));
-          ok = wait_phase(q_full(1), 0, abort_flag, p.err);
+          mma_commit_elect(s_full(0));
+          ok = warp_wait_phase(q_full(1), 0, abort_flag, p.err);
         }
         if (ok) {
           tc_fence_after();
           issue_qk<D>(tmem + (C::kTmemS + 128), sQ[1], sKV(ks));
-          mma_commit(s_full(1));
-          mma_commit(kv_empty(ks));
+          mma_commit_elect(s_full(1));
+          mma_commit_elect(kv_empty(ks));
         }
         while (ok) {
           const int vs = n % C::kStages;
-          ok = wait_phase(kv_full(vs), (n / C::kStages) & 1, abort_flag, p.err);
+          VIDATTN_TR(0, t, 0);
+          ok = warp_wait_phase(kv_full(vs), (n / C::kStages) & 1, abort_flag, p.err);
           ++n;
           if (!ok) break;
           const int jn = sched.tile(t + 1, j);
-          ok = wait_phase(p_full(0), t & 1, abort_flag, p.err);
+          ok = warp_wait_phase(p_full(0), t & 1, abort_flag, p.err);
+          VIDATTN_TR(0, t, 3);
           if (!ok) break;
           tc_fence_after();
           issue_pv<D>(tmem + C::kTmemO, tmem + C::kTmemS, sKV(vs), t > 0);
-          mma_commit(o_full(0));
+          mma_commit_elect(o_full(0));
+          VIDATTN_TR(0, t, 4);
           int ks2 = 0;
           if (jn < n_kv) {
             ks2 = n % C::kStages;
-            ok = wait_phase(kv_full(ks2), (n / C::kStages) & 1, abort_flag, p.err);
+            ok = warp_wait_phase(kv_full(ks2), (n / C::kStages) & 1, abort_flag, p.err);
             ++n;
             if (!ok) break;
             tc_fence_after();
             issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(ks2));
-            mma_commit(s_full(0));
+            mma_commit_elect(s_full(0));
+            VIDATTN_TR(0, t, 2);
           }
-          ok = wait_phase(p_full(1), t & 1, abort_flag, p.err);
+          ok = warp_wait_phase(p_full(1), t & 1, abort_flag, p.err);
+          VIDATTN_TR(0, t, 7);
           if (!ok) break;
           tc_fence_after();
           issue_pv<D>(tmem + (C::kTmemO + D), tmem + (C::kTmemS + 128), sKV(vs), t > 0);
-          mma_commit(o_full(1));
-          mma_commit(kv_empty(vs));
+          mma_commit_elect(o_full(1));
+          mma_commit_elect(kv_empty(vs));
           if (jn >= n_kv) break;
           issue_qk<D>(tmem + (C::kTmemS + 128), sQ[1], sKV(ks2));
-          mma_commit(s_full(1));
-          mma_commit(kv_empty(ks2));
+          mma_commit_elect(s_full(1));
+          mma_commit_elect(kv_empty(ks2));
+          VIDATTN_TR(0, t, 8);
           j = jn;
           ++t;
         }
         // Every MMA issued above has finished before TMEM is released.
-        mma_commit(drain_bar);
+        mma_commit_elect(drain_bar);
         volatile int never = 0;
-        wait_phase(drain_bar, 0, &never, p.err);
+        warp_wait_phase(drain_bar, 0, &never, p.err);
       }
     }
     __syncwarp();
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+    if constexpr (D == 128) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+    } else {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory");
+    }
     // ------------------------------------------------------------ softmax
     const int qi = warp >> 2;                       // which Q tile
     const int r = ((warp & 3) << 5) + lane;         // row in the tile = TMEM lane
@@ -493,6 +616,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kTmemS + 128u * qi;
     const uint32_t tO = tmem + lane_off + C::kTmemO + uint32_t(D) * qi;
+    const uint32_t tP = tmem + lane_off + C::kTmemP + C::kPStride * qi;
     int4 my_qs;
     const KvSched sched{listed ? tile_list : nullptr, n_list,
                         make_walk(p, b, blockIdx.x, qi, &my_qs)};
@@ -515,99 +639,185 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       const bool slow = masked || !(c > 0.f);
+      VIDATTN_TR(1 + qi, t, 0);
       ok = warp_wait_phase(s_full(qi), t & 1, abort_flag, p.err);
+      VIDATTN_TR(1 + qi, t, 1);
       if (!ok) break;
       tc_fence_after();
-      // P = 2^(c*s - m_run) for this tile, rounded to bf16 into pk; rs = its
-      // row sum in fp32.  Softmax does not depend on the offset m_run, so after
-      // a row's first tile the running offset is used as it stands ("stale"
-      // path, no max).  The offset only has to keep every exponential finite:
-      // if the tile's sum exceeds 2^32 the row takes the exact path instead,
-      // which computes the tile max, moves m_run up (rescaling O and l), and
-      // redoes the exponentials.  The exact path also serves masked tiles,
-      // a row's first tile, and scale <= 0.
-      float rs = 0.f, alpha = 1.f;
-      bool rescale = false;
-      // warp-uniform choice: the stale path only if every row of the warp can take it
-      bool exact = __any_sync(0xffffffffu, slow || (m_run == -INFINITY));
-      if (!exact) {
+      if constexpr (C::kSepP) {
+        // S row into registers, then S's columns are released to the MMA warp.
         float s[kBN];
-        uint32_t pk[2][32];
         load_s_row(tS, s);
-        rs = exp_tile<kEmu>(s, c, m_run, pk);
-        exact = __any_sync(0xffffffffu, !(rs <= kStaleSumLimit));
+        tc_fence_before();
+        mbar_arrive(s_free(qi));
+        VIDATTN_TR(1 + qi, t, 2);
+        uint32_t pk[2][32];
+        float rs = 0.f, alpha = 1.f;
+        bool rescale = false;
+        // running-offset path first (see the aliased-P branch below); the
+        // exact path works on the registers, since S may be overwritten now
+        bool exact = __any_sync(0xffffffffu, slow || (m_run == -INFINITY));
         if (!exact) {
-          tmem_st32(tS, pk[0]);
-          tmem_st32(tS + 32, pk[1]);
+          rs = exp_tile<kEmu>(s, c, m_run, pk);
+          exact = __any_sync(0xffffffffu, !(rs <= kStaleSumLimit));
         }
-      }
-      if (exact) {
-        // Two passes over the tile, 32 columns at a time, straight from
-        // tensor memory (S is intact: no P has been written yet).
-        const int j0 = j * kBN;
-        auto allowed = [&](int x) {
-          bool valid = (j0 + x) < p.S_kv;
-          if (has_seg && valid) valid = __ldg(seg_kv_b + j0 + x) == my_seg;
-          return valid;
-        };
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int k = 0; k < 4; ++k) {
-          uint32_t r[32];
-          tmem_ld32(tS + 32 * k, r);
-          tmem_ld_wait();
-          reg_fence(r);
+        if (exact) {
+          float tile_max;
+          if (!slow) {
+            tile_max = row_max(s) * c;
+          } else {
+            const int j0 = j * kBN;
+            float mx = -INFINITY;
 #pragma unroll
-          for (int x = 0; x < 32; ++x)
-            mx = fmaxf(mx, allowed(32 * k + x) ? __uint_as_float(r[x]) * c : -INFINITY);
-        }
-        const float m_new = fmaxf(m_run, mx);
-        rescale = (m_new - m_run) > kRescaleThreshold;   // false for -inf - -inf
-        if (rescale) {
-          alpha = ex2(m_run - m_new);   // 0 when m_run is -inf
-          m_run = m_new;
-        }
-        const float msub = (m_run == -INFINITY) ? 0.f : m_run;
-        // P chunk k (keys 32k..32k+31) lands in columns [16k, 16k+16), which
-        // hold S columns already read: chunks are processed in order.
-#pragma unroll 1
-        for (int k = 0; k < 4; ++k) {
-          uint32_t r[32], w[16];
-          tmem_ld32(tS + 32 * k, r);
-          tmem_ld_wait();
-          reg_fence(r);
-#pragma unroll
-          for (int x = 0; x < 32; x += 2) {
-            const float e0 = allowed(32 * k + x) ? ex2(__uint_as_float(r[x]) * c - msub) : 0.f;
-            const float e1 =
-                allowed(32 * k + x + 1) ? ex2(__uint_as_float(r[x + 1]) * c - msub) : 0.f;
-            rs += e0 + e1;
-            w[x >> 1] = pack_bf16x2(e0, e1);
+            for (int x = 0; x < kBN; ++x) {
+              bool valid = (j0 + x) < p.S_kv;
+              if (has_seg && valid) valid = __ldg(seg_kv_b + j0 + x) == my_seg;
+              s[x] = valid ? s[x] * c : -INFINITY;
+              mx = fmaxf(mx, s[x]);
+            }
+            tile_max = mx;
           }
-          tmem_st16(tS + 16 * k, w);
-        }
-      }
-      l_run = l_run * alpha + rs;
-      tmem_st_wait();
-      // Rescale this tile's O rows before the next P.V accumulates into them.
-      if (__any_sync(0xffffffffu, rescale && t > 0)) {
-        ok = warp_wait_phase(o_full(qi), (t - 1) & 1, abort_flag, p.err);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int k = 0; k < D / 32; ++k) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * k, o);
-          tmem_ld_wait();
-          reg_fence(o);
+          const float m_new = fmaxf(m_run, tile_max);
+          rescale = (m_new - m_run) > kRescaleThreshold;
+          if (rescale) {
+            alpha = ex2(m_run - m_new);
+            m_run = m_new;
+          }
+          const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+          if (!slow) {
+            rs = exp_tile<kEmu>(s, c, msub, pk);
+          } else {
+            float r4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-          tmem_st32(tO + 32 * k, o);
+            for (int x = 0; x < kBN; x += 2) {
+              const float e0 = ex2(s[x] - msub);
+              const float e1 = ex2(s[x + 1] - msub);
+              r4[(x >> 1) & 3] += e0 + e1;
+              pk[x >> 6][(x >> 1) & 31] = pack_bf16x2(e0, e1);
+            }
+            rs = (r4[0] + r4[1]) + (r4[2] + r4[3]);
+          }
+        }
+        l_run = l_run * alpha + rs;
+        VIDATTN_TR(1 + qi, t, 3);
+        // The previous P V of this tile has read P's columns and finished
+        // accumulating O: P may be overwritten and O rescaled.
+        if (t > 0) {
+          ok = warp_wait_phase(o_full(qi), (t - 1) & 1, abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        VIDATTN_TR(1 + qi, t, 4);
+        tmem_st32(tP, pk[0]);
+        tmem_st32(tP + 32, pk[1]);
+        if (__any_sync(0xffffffffu, rescale && t > 0)) {
+#pragma unroll 1
+          for (int k = 0; k < D / 32; ++k) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * k, o);
+            tmem_ld_wait();
+            reg_fence(o);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            tmem_st32(tO + 32 * k, o);
+          }
         }
         tmem_st_wait();
+      } else {
+        // P = 2^(c*s - m_run) for this tile, rounded to bf16 into pk; rs = its
+        // row sum in fp32.  Softmax does not depend on the offset m_run, so after
+        // a row's first tile the running offset is used as it stands ("stale"
+        // path, no max).  The offset only has to keep every exponential finite:
+        // if the tile's sum exceeds 2^32 the row takes the exact path instead,
+        // which computes the tile max, moves m_run up (rescaling O and l), and
+        // redoes the exponentials.  The exact path also serves masked tiles,
+        // a row's first tile, and scale <= 0.
+        float rs = 0.f, alpha = 1.f;
+        bool rescale = false;
+        // warp-uniform choice: the stale path only if every row of the warp can take it
+        bool exact = __any_sync(0xffffffffu, slow || (m_run == -INFINITY));
+        if (!exact) {
+          float s[kBN];
+          uint32_t pk[2][32];
+          load_s_row(tS, s);
+          VIDATTN_TR(1 + qi, t, 2);
+          rs = exp_tile<kEmu>(s, c, m_run, pk);
+          VIDATTN_TR(1 + qi, t, 3);
+          exact = __any_sync(0xffffffffu, !(rs <= kStaleSumLimit));
+          if (!exact) {
+            tmem_st32(tS, pk[0]);
+            tmem_st32(tS + 32, pk[1]);
+          }
+        }
+        if (exact) {
+          // Two passes over the tile, 32 columns at a time, straight from
+          // tensor memory (S is intact: no P has been written yet).
+          const int j0 = j * kBN;
+          auto allowed = [&](int x) {
+            bool valid = (j0 + x) < p.S_kv;
+            if (has_seg && valid) valid = __ldg(seg_kv_b + j0 + x) == my_seg;
+            return valid;
+          };
+          float mx = -INFINITY;
+  #pragma unroll 1
+          for (int k = 0; k < 4; ++k) {
+            uint32_t r[32];
+            tmem_ld32(tS + 32 * k, r);
+            tmem_ld_wait();
+            reg_fence(r);
+  #pragma unroll
+            for (int x = 0; x < 32; ++x)
+              mx = fmaxf(mx, allowed(32 * k + x) ? __uint_as_float(r[x]) * c : -INFINITY);
+          }
+          const float m_new = fmaxf(m_run, mx);
+          rescale = (m_new - m_run) > kRescaleThreshold;   // false for -inf - -inf
+          if (rescale) {
+            alpha = ex2(m_run - m_new);   // 0 when m_run is -inf
+            m_run = m_new;
+          }
+          const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+          // P chunk k (keys 32k..32k+31) lands in columns [16k, 16k+16), which
+          // hold S columns already read: chunks are processed in order.
+  #pragma unroll 1
+          for (int k = 0; k < 4; ++k) {
+            uint32_t r[32], w[16];
+            tmem_ld32(tS + 32 * k, r);
+            tmem_ld_wait();
+            reg_fence(r);
+  #pragma unroll
+            for (int x = 0; x < 32; x += 2) {
+              const float e0 = allowed(32 * k + x) ? ex2(__uint_as_float(r[x]) * c - msub) : 0.f;
+              const float e1 =
+                  allowed(32 * k + x + 1) ? ex2(__uint_as_float(r[x + 1]) * c - msub) : 0.f;
+              rs += e0 + e1;
+              w[x >> 1] = pack_bf16x2(e0, e1);
+            }
+            tmem_st16(tS + 16 * k, w);
+          }
+        }
+        l_run = l_run * alpha + rs;
+        tmem_st_wait();
+        // Rescale this tile's O rows before the next P.V accumulates into them.
+        if (__any_sync(0xffffffffu, rescale && t > 0)) {
+          ok = warp_wait_phase(o_full(qi), (t - 1) & 1, abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+  #pragma unroll 1
+          for (int k = 0; k < D / 32; ++k) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * k, o);
+            tmem_ld_wait();
+            reg_fence(o);
+  #pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            tmem_st32(tO + 32 * k, o);
+          }
+          tmem_st_wait();
+        }
       }
       tc_fence_before();
       mbar_arrive(p_full(qi));
+      VIDATTN_TR(1 + qi, t, 5);
     }
 
     // ------------------------------------------------------------ epilogue

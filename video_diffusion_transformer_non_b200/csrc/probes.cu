@@ -52,19 +52,24 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(slot);
 
+  // Warp 0 issues, converged: issue_qk / issue_pv elect one lane per MMA,
+  // and the commits elect the same lane (a commit tracks its own thread's MMAs).
   bool ok = true;
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar_load, 3 * C::kTileBytes);
-    for (int s = 0; s < C::kSub; ++s) {
-      tma_load_3d(sQ + s * C::kSubBytes, &tm_q, bar_load, s * 64, 0, 0);
-      tma_load_3d(sK + s * C::kSubBytes, &tm_k, bar_load, s * 64, 0, 0);
-      tma_load_3d(sV + s * C::kSubBytes, &tm_v, bar_load, s * 64, 0, 0);
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_load, 3 * C::kTileBytes);
+      for (int s = 0; s < C::kSub; ++s) {
+        tma_load_3d(sQ + s * C::kSubBytes, &tm_q, bar_load, s * 64, 0, 0);
+        tma_load_3d(sK + s * C::kSubBytes, &tm_k, bar_load, s * 64, 0, 0);
+        tma_load_3d(sV + s * C::kSubBytes, &tm_v, bar_load, s * 64, 0, 0);
+      }
     }
-    ok = wait_phase(bar_load, 0, abort_flag, status, 100000000ull);
+    __syncwarp();
+    ok = warp_wait_phase(bar_load, 0, abort_flag, status, 100000000ull);
     if (ok) {
       tc_fence_after();
       issue_qk<D>(tmem + 0, sQ, sK);
-      mma_commit(bar_mma);
+      mma_commit_elect(bar_mma);
     }
   }
   ok = __syncthreads_and(ok);
@@ -93,10 +98,10 @@ __global__ void __launch_bounds__(128, 1)
   }
   tc_fence_before();
   ok = __syncthreads_and(ok);
-  if (ok && threadIdx.x == 0) {
+  if (ok && warp == 0) {
     tc_fence_after();
     issue_pv<D>(tmem + 384, tmem + 256, sV, false);
-    mma_commit(bar_mma);
+    mma_commit_elect(bar_mma);
   }
   ok = ok && wait_phase(bar_mma, 1, abort_flag, status, 100000000ull);
   ok = __all_sync(0xffffffffu, ok);

@@ -19,6 +19,11 @@
 
 namespace vidattn {
 
+#ifdef VIDATTN_TRACE
+// Trace builds only: the buffer vidattn_trace_set() names (4 x 64 x 16 u64).
+unsigned long long* g_trace = nullptr;
+#endif
+
 // Device error word: kernels OR error bits into it (see kErrTimeout).
 __device__ int g_device_error = 0;
 
@@ -224,6 +229,9 @@ int launch_fwd(const void* q, const void* k, const void* v, const int32_t* seg_q
   p.n_q_tiles = (S_q + kBM - 1) / kBM;
   p.n_kv_tiles = (S_kv + kBN - 1) / kBN;
   p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+#ifdef VIDATTN_TRACE
+  p.trace = g_trace;
+#endif
   dim3 grid((S_q + 2 * kBM - 1) / (2 * kBM), H, B);
   FwdKernel kernel = fwd_variant<D>(emu_index(D));
   kernel<<<grid, kFwdThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
@@ -436,3 +444,9 @@ VIDATTN_API void vidattn_release(void) {
 }
 
 }  // extern "C"
+
+#ifdef VIDATTN_TRACE
+// Trace builds only (not part of the product ABI): where the next launches
+// write their timeline stamps; NULL stops tracing.
+extern "C" VIDATTN_API void vidattn_trace_set(unsigned long long* buffer) { g_trace = buffer; }
+#endif
