@@ -92,8 +92,9 @@ FwdKernel fwd_variant(int e) {
     default: return vidattn_fwd_kernel<D, 8>;
   }
 }
-// Default share of exponentials moved off the MUFU unit: at D = 128 the
-// exp2 work per key tile equals the tensor-core time, at D = 64 twice it.
+// Default share of exponentials moved off the MUFU unit (measured best on
+// B200: 4 of 16 at D = 128, 2 of 16 at D = 64, where the FMA-pipe version's
+// extra instructions cost more than the MUFU time they save).
 // VIDATTN_EMU (0, 2, 4, 6 or 8 per 16 keys) overrides, for experiments.
 int emu_index(int D) {
   static const int forced = [] {
@@ -105,7 +106,7 @@ int emu_index(int D) {
     return -1;
   }();
   if (forced >= 0) return forced;
-  return D == 128 ? 2 : 4;
+  return D == 128 ? 2 : 1;
 }
 std::mutex g_mu;
 std::map<int, DeviceInfo> g_devices;
