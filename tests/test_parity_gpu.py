@@ -109,6 +109,35 @@ def test_peaked_softmax_with_head_scaling():
     check_all_rows(c, what="peaked")
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("with_ids", [False, True])
+@pytest.mark.parametrize("pattern", ["per_tile", "within_tile"])
+def test_running_offset_overflow_takes_exact_path(D, with_ids, pattern):
+    """Keys scaled so that scores grow along the sequence: the offset a row
+    takes from its first key tile goes stale by far more than 2^32 in P, and
+    the kernel must fall back to the exact path (tile max, rescale of O and
+    the row sum) and still match the oracle.  per_tile: 128-key tiles scaled
+    0.05x .. 16x (the whole tile overflows).  within_tile: 64-key halves
+    scaled so that only the second half of a tile overflows."""
+    B, H, S_q, S_kv = 1, 2, 300, 640
+    rng = np.random.Generator(np.random.PCG64(46 + D))
+    q = rng.standard_normal((B, H, S_q, D), dtype=np.float32)
+    k = rng.standard_normal((B, H, S_kv, D), dtype=np.float32)
+    v = rng.standard_normal((B, H, S_kv, D), dtype=np.float32)
+    if pattern == "per_tile":
+        blocks, factors = 128, [0.05, 0.5, 2.0, 8.0, 16.0]
+    else:
+        blocks, factors = 64, [0.05, 0.05, 0.5, 0.5, 2.0, 2.0, 2.0, 8.0, 8.0, 16.0]
+    for j, f in enumerate(factors):
+        k[:, :, blocks * j:blocks * (j + 1)] *= np.float32(f)
+    c = dict(q=wl.f32_to_bf16_bits(q), k=wl.f32_to_bf16_bits(k), v=wl.f32_to_bf16_bits(v),
+             seg_q=None, seg_kv=None, scale=1.0 / np.sqrt(D))
+    if with_ids:   # one id everywhere: the listed-tile path, same result
+        c["seg_q"] = np.zeros((B, S_q), np.int32)
+        c["seg_kv"] = np.zeros((B, S_kv), np.int32)
+    check_all_rows(c, what=f"stale offset {pattern} D{D} ids={with_ids}")
+
+
 def test_scale_zero_with_segments_gives_segment_means():
     c = runs_case(1, 2, ((200, 0), (100, 1), (20, 2)), 128, 40)
     check_all_rows(c, scale=0.0, what="scale 0 + ids")

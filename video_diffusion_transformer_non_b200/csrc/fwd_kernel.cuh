@@ -485,9 +485,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const bool more = jn < n_kv;
           const int kn = 2 * (t + 1), vi = 2 * t + 1;
           VIDATTN_TR(0, t, 0);
+          // both tiles' data first (see the aliased loop)
+          ok = warp_wait_phase(kv_full(stage(vi)), par(vi), abort_flag, p.err);
+          if (ok && more) ok = warp_wait_phase(kv_full(stage(kn)), par(kn), abort_flag, p.err);
+          if (!ok) break;
           if (more) {
-            ok = warp_wait_phase(kv_full(stage(kn)), par(kn), abort_flag, p.err) &&
-                 warp_wait_phase(s_free(0), t & 1, abort_flag, p.err);
+            ok = warp_wait_phase(s_free(0), t & 1, abort_flag, p.err);
             VIDATTN_TR(0, t, 1);
             if (!ok) break;
             tc_fence_after();
@@ -495,8 +498,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mma_commit_elect(s_full(0));
             VIDATTN_TR(0, t, 2);
           }
-          ok = warp_wait_phase(kv_full(stage(vi)), par(vi), abort_flag, p.err) &&
-               warp_wait_phase(p_full(0), t & 1, abort_flag, p.err);
+          ok = warp_wait_phase(p_full(0), t & 1, abort_flag, p.err);
           VIDATTN_TR(0, t, 3);
           if (!ok) break;
           tc_fence_after();
@@ -559,6 +561,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ++n;
           if (!ok) break;
           const int jn = sched.tile(t + 1, j);
+          // Check that K_{t+1} has landed now, while this warp waits anyway,
+          // instead of between dependent MMAs (an mbarrier read is slow while
+          // a shared-memory-bound Q K^T runs).
+          int ks2 = 0;
+          if (jn < n_kv) {
+            ks2 = n % C::kStages;
+            ok = warp_wait_phase(kv_full(ks2), (n / C::kStages) & 1, abort_flag, p.err);
+            ++n;
+            if (!ok) break;
+          }
           ok = warp_wait_phase(p_full(0), t & 1, abort_flag, p.err);
           VIDATTN_TR(0, t, 3);
           if (!ok) break;
@@ -566,12 +578,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           issue_pv<D>(tmem + C::kTmemO, tmem + C::kTmemS, sKV(vs), t > 0);
           mma_commit_elect(o_full(0));
           VIDATTN_TR(0, t, 4);
-          int ks2 = 0;
           if (jn < n_kv) {
-            ks2 = n % C::kStages;
-            ok = warp_wait_phase(kv_full(ks2), (n / C::kStages) & 1, abort_flag, p.err);
-            ++n;
-            if (!ok) break;
             tc_fence_after();
             issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(ks2));
             mma_commit_elect(s_full(0));
@@ -751,7 +758,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         if (exact) {
           // Two passes over the tile, 32 columns at a time, straight from
-          // tensor memory (S is intact: no P has been written yet).
+          // tensor memory (S is intact: no P has been written yet).  The sum
+          // restarts: a failed running-offset attempt leaves its sum in rs.
+          rs = 0.f;
           const int j0 = j * kBN;
           auto allowed = [&](int x) {
             bool valid = (j0 + x) < p.S_kv;

@@ -74,7 +74,30 @@ struct DeviceInfo {
   bool checked = false;
   bool ok = false;
   uint32_t attrs_set = 0;   // bit (kernel variant index) once its smem limit is raised
+  int* err = nullptr;       // device address of g_device_error on this device
 };
+
+// Recently encoded tensor maps (per device): a call on the same buffers and
+// shape reuses them instead of encoding three descriptors again.
+struct MapKey {
+  int dev;
+  const void* ptr;
+  int64_t BH, S;
+  int D;
+  bool operator==(const MapKey& o) const {
+    return dev == o.dev && ptr == o.ptr && BH == o.BH && S == o.S && D == o.D;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  uint64_t stamp;
+};
+constexpr int kMapCacheSize = 16;
+MapEntry g_map_cache[kMapCacheSize];
+int g_map_used = 0;
+uint64_t g_map_clock = 0;
+std::mutex g_map_mu;
 
 using FwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                            const FwdParams);
@@ -132,6 +155,12 @@ int ensure_device(int* dev_out) {
     info.ok = (major == 10 && minor == 0);
   }
   if (!info.ok) return VIDATTN_ERR_NO_DEVICE;
+  if (info.err == nullptr) {
+    void* e = nullptr;
+    if (cudaGetSymbolAddress(&e, g_device_error) != cudaSuccess || e == nullptr)
+      return VIDATTN_ERR_CUDA;
+    info.err = static_cast<int*>(e);
+  }
   if (info.attrs_set == 0) {
     for (int e = 0; e < kNumEmu; ++e) {
       if (cudaFuncSetAttribute(fwd_variant<64>(e), cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -182,6 +211,35 @@ int noalloc_scratch(int dev, int4** out) {
   return VIDATTN_OK;
 }
 
+int* device_error_word(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_devices[dev].err;
+}
+
+// Tensor map of bf16 [BH, S, D] at ptr on dev, from the cache when present.
+bool cached_map(int dev, const void* ptr, int64_t BH, int64_t S, int D, CUtensorMap* out) {
+  const MapKey key{dev, ptr, BH, S, D};
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  for (int i = 0; i < g_map_used; ++i) {
+    if (g_map_cache[i].key == key) {
+      g_map_cache[i].stamp = ++g_map_clock;
+      *out = g_map_cache[i].map;
+      return true;
+    }
+  }
+  if (!encode_bhsd(out, ptr, BH, S, D)) return false;
+  int slot = g_map_used;
+  if (g_map_used < kMapCacheSize) {
+    ++g_map_used;
+  } else {
+    slot = 0;
+    for (int i = 1; i < kMapCacheSize; ++i)
+      if (g_map_cache[i].stamp < g_map_cache[slot].stamp) slot = i;
+  }
+  g_map_cache[slot] = MapEntry{key, *out, ++g_map_clock};
+  return true;
+}
+
 inline bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
@@ -202,7 +260,7 @@ int check_args(const void* q, const void* k, const void* v, const int32_t* seg_q
 }
 
 template <int D>
-int launch_fwd(const void* q, const void* k, const void* v, const int32_t* seg_q,
+int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32_t* seg_q,
                const int32_t* seg_kv, const int4* q_sum, const int4* kv_sum, void* out,
                float* lse, int B, int H, int S_q, int S_kv, float scale, cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
@@ -210,8 +268,8 @@ int launch_fwd(const void* q, const void* k, const void* v, const int32_t* seg_q
   // With no keys the K/V maps are never read; they are encoded over q.
   const void* kp = S_kv > 0 ? k : q;
   const void* vp = S_kv > 0 ? v : q;
-  if (!encode_bhsd(&tq, q, BH, S_q, D) || !encode_bhsd(&tk, kp, BH, S_kv, D) ||
-      !encode_bhsd(&tv, vp, BH, S_kv, D))
+  if (!cached_map(dev, q, BH, S_q, D, &tq) || !cached_map(dev, kp, BH, S_kv, D, &tk) ||
+      !cached_map(dev, vp, BH, S_kv, D, &tv))
     return VIDATTN_ERR_CUDA;
   FwdParams p{};
   p.seg_q = seg_q;
@@ -220,10 +278,7 @@ int launch_fwd(const void* q, const void* k, const void* v, const int32_t* seg_q
   p.kv_sum = kv_sum;
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;
-  int* err = nullptr;
-  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_device_error) != cudaSuccess)
-    return VIDATTN_ERR_CUDA;
-  p.err = err;
+  p.err = device_error_word(dev);
   p.H = H;
   p.S_q = S_q;
   p.S_kv = S_kv;
@@ -318,9 +373,9 @@ VIDATTN_API int vidattn_fwd(const void* q, const void* k, const void* v, const i
     if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
   }
   if (D == 64)
-    return launch_fwd<64>(q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
+    return launch_fwd<64>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
                           stream);
-  return launch_fwd<128>(q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
+  return launch_fwd<128>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
                          stream);
 }
 
@@ -409,9 +464,9 @@ VIDATTN_API int vidattn_fwd_noalloc(const void* q, const void* k, const void* v,
     if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
   }
   if (D == 64)
-    return launch_fwd<64>(q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
+    return launch_fwd<64>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
                           stream);
-  return launch_fwd<128>(q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
+  return launch_fwd<128>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
                          stream);
 }
 
