@@ -8,7 +8,8 @@ The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, OpenMP over rows);
 this module compiles it with gcc and marshals numpy arrays through ctypes.
 What it computes, with citations, is written at the top of ``attn_oracle.c``:
 exact softmax(scale * Q K^T masked by segment-id equality) V, plus the natural
-log-sum-exp of each row, with empty rows giving out = 0 and lse = -inf.
+log-sum-exp of each row, with empty rows giving out = 0 and lse = -inf; with
+causal=True a key is also limited to j <= i + (S_kv - S_q).
 
 Inputs are bf16 bit patterns as ``numpy.uint16`` arrays in [B,H,S,D] order and
 int32 segment ids in [B,S] order (or None for a single segment).
@@ -47,12 +48,13 @@ def _load():
         p = ctypes.c_void_p
         L = ctypes.c_long
         lib.oracle_attn_fwd_f64.argtypes = [p, p, p, p, p, p, p, L, L, L, L, L,
-                                            ctypes.c_double, ctypes.c_int]
+                                            ctypes.c_double, ctypes.c_int, ctypes.c_int]
         lib.oracle_attn_fwd_f64.restype = ctypes.c_int
         lib.oracle_attn_rows_f64.argtypes = [p, p, p, p, p, p, L, p, p, L, L, L, L, L,
-                                             ctypes.c_double, ctypes.c_int]
+                                             ctypes.c_double, ctypes.c_int, ctypes.c_int]
         lib.oracle_attn_rows_f64.restype = ctypes.c_int
-        lib.oracle_attn_probs_f64.argtypes = [p, p, p, p, p, L, L, L, L, L, ctypes.c_double]
+        lib.oracle_attn_probs_f64.argtypes = [p, p, p, p, p, L, L, L, L, L, ctypes.c_double,
+                                              ctypes.c_int]
         lib.oracle_attn_probs_f64.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -79,7 +81,7 @@ def _check_inputs(q, k, v, seg_q, seg_kv):
     return B, H, S_q, S_kv, D
 
 
-def attn_fwd(q, k, v, seg_q=None, seg_kv=None, scale=None, nthreads=0):
+def attn_fwd(q, k, v, seg_q=None, seg_kv=None, scale=None, nthreads=0, causal=False):
     """All rows.  Returns (out float64 [B,H,S_q,D], lse float64 [B,H,S_q])."""
     B, H, S_q, S_kv, D = _check_inputs(q, k, v, seg_q, seg_kv)
     if scale is None:
@@ -88,13 +90,13 @@ def attn_fwd(q, k, v, seg_q=None, seg_kv=None, scale=None, nthreads=0):
     lse = np.empty((B, H, S_q), np.float64)
     rc = _load().oracle_attn_fwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv),
                                      _ptr(out), _ptr(lse), B, H, S_q, S_kv, D,
-                                     float(scale), int(nthreads))
+                                     float(scale), int(bool(causal)), int(nthreads))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd_f64 failed with code {rc}")
     return out, lse
 
 
-def attn_rows(q, k, v, rows, seg_q=None, seg_kv=None, scale=None, nthreads=0):
+def attn_rows(q, k, v, rows, seg_q=None, seg_kv=None, scale=None, nthreads=0, causal=False):
     """Selected rows.  rows: int64 [n,3] of (b, h, i).
     Returns (out float64 [n,D], lse float64 [n])."""
     B, H, S_q, S_kv, D = _check_inputs(q, k, v, seg_q, seg_kv)
@@ -106,13 +108,14 @@ def attn_rows(q, k, v, rows, seg_q=None, seg_kv=None, scale=None, nthreads=0):
     lse = np.empty((n,), np.float64)
     rc = _load().oracle_attn_rows_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv),
                                       _ptr(rows), n, _ptr(out), _ptr(lse),
-                                      B, H, S_q, S_kv, D, float(scale), int(nthreads))
+                                      B, H, S_q, S_kv, D, float(scale), int(bool(causal)),
+                                      int(nthreads))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_rows_f64 failed with code {rc}")
     return out, lse
 
 
-def attn_probs(q, k, seg_q=None, seg_kv=None, scale=None):
+def attn_probs(q, k, seg_q=None, seg_kv=None, scale=None, causal=False):
     """Softmax weights [B,H,S_q,S_kv] (small inputs only); masked entries are 0."""
     B, H, S_q, D = q.shape
     S_kv = k.shape[2]
@@ -121,7 +124,8 @@ def attn_probs(q, k, seg_q=None, seg_kv=None, scale=None):
         scale = 1.0 / np.sqrt(D)
     probs = np.empty((B, H, S_q, S_kv), np.float64)
     rc = _load().oracle_attn_probs_f64(_ptr(q), _ptr(k), _ptr(seg_q), _ptr(seg_kv),
-                                       _ptr(probs), B, H, S_q, S_kv, D, float(scale))
+                                       _ptr(probs), B, H, S_q, S_kv, D, float(scale),
+                                       int(bool(causal)))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_probs_f64 failed with code {rc}")
     return probs

@@ -29,6 +29,12 @@
  * segment ids are equal; a row that sees no key gets out = 0 and lse = -inf;
  * lse is the natural log over the scaled logits of the allowed keys.
  *
+ * Causal variant (same paper, §3.1, Cosmos paragraph: a backbone whose
+ * "understanding" pathway attends causally): with causal != 0 a key is
+ * allowed only if, in addition, j <= i + (S_kv - S_q), i.e. query i sees
+ * the keys up to its own position, the last query aligned with the last
+ * key.  The set A_i above gains this condition; nothing else changes.
+ *
  * Parallelism: OpenMP over independent rows only; the arithmetic of a row is
  * the serial loop above.  Build without -ffast-math.
  */
@@ -48,23 +54,29 @@ static double bf16_bits_to_double(uint16_t bits) {
   return (double)f;
 }
 
+/* Is key j visible to query i?  (segment equality; causal limit) */
+static int key_allowed(const int32_t* seg_q, const int32_t* seg_kv, long S_q, long S_kv,
+                       long b, long i, long j, int causal) {
+  if (seg_q != NULL && seg_kv[b * S_kv + j] != seg_q[b * S_q + i]) return 0;
+  if (causal && j > i + (S_kv - S_q)) return 0;
+  return 1;
+}
+
 /* One output row (b, h, i).  s_scratch holds S_kv doubles. */
 static void oracle_row(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                        const int32_t* seg_q, const int32_t* seg_kv,
-                       long H, long S_q, long S_kv, long D, double scale,
+                       long H, long S_q, long S_kv, long D, double scale, int causal,
                        long b, long h, long i, double* s_scratch,
                        double* out_row, double* lse_out) {
   const uint16_t* qi = q + ((b * H + h) * S_q + i) * D;
   const uint16_t* kb = k + (b * H + h) * S_kv * D;
   const uint16_t* vb = v + (b * H + h) * S_kv * D;
-  const int has_seg = (seg_q != NULL);
-  const int32_t sid = has_seg ? seg_q[b * S_q + i] : 0;
 
   /* scores of the allowed keys, and their maximum */
   double m = -INFINITY;
   long n_allowed = 0;
   for (long j = 0; j < S_kv; ++j) {
-    int allowed = !has_seg || (seg_kv[b * S_kv + j] == sid);
+    int allowed = key_allowed(seg_q, seg_kv, S_q, S_kv, b, i, j, causal);
     if (!allowed) { s_scratch[j] = NAN; continue; }
     double dot = 0.0;
     for (long d = 0; d < D; ++d)
@@ -84,7 +96,7 @@ static void oracle_row(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   /* softmax weights, their sum, and the weighted sum of values */
   double l = 0.0;
   for (long j = 0; j < S_kv; ++j) {
-    int allowed = !has_seg || (seg_kv[b * S_kv + j] == sid);
+    int allowed = key_allowed(seg_q, seg_kv, S_q, S_kv, b, i, j, causal);
     if (!allowed) continue;
     double e = exp(s_scratch[j] - m);
     l += e;
@@ -107,7 +119,7 @@ int oracle_attn_fwd_f64(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         const int32_t* seg_q, const int32_t* seg_kv,
                         double* out, double* lse,
                         long B, long H, long S_q, long S_kv, long D,
-                        double scale, int nthreads) {
+                        double scale, int causal, int nthreads) {
   if (check_shape(B, H, S_q, S_kv, D)) return 1;
   if ((seg_q == NULL) != (seg_kv == NULL)) return 1;
   long n_rows = B * H * S_q;
@@ -129,7 +141,7 @@ int oracle_attn_fwd_f64(const uint16_t* q, const uint16_t* k, const uint16_t* v,
         long i = r % S_q;
         long h = (r / S_q) % H;
         long b = r / (S_q * H);
-        oracle_row(q, k, v, seg_q, seg_kv, H, S_q, S_kv, D, scale, b, h, i,
+        oracle_row(q, k, v, seg_q, seg_kv, H, S_q, S_kv, D, scale, causal, b, h, i,
                    s_scratch, out + r * D, lse + r);
       }
       free(s_scratch);
@@ -145,7 +157,7 @@ int oracle_attn_rows_f64(const uint16_t* q, const uint16_t* k, const uint16_t* v
                          const int64_t* rows, long n_rows,
                          double* out_rows, double* lse_rows,
                          long B, long H, long S_q, long S_kv, long D,
-                         double scale, int nthreads) {
+                         double scale, int causal, int nthreads) {
   if (check_shape(B, H, S_q, S_kv, D) || n_rows < 0) return 1;
   if ((seg_q == NULL) != (seg_kv == NULL)) return 1;
   for (long r = 0; r < n_rows; ++r) {
@@ -168,7 +180,7 @@ int oracle_attn_rows_f64(const uint16_t* q, const uint16_t* k, const uint16_t* v
     } else {
 #pragma omp for schedule(dynamic, 1)
       for (long r = 0; r < n_rows; ++r)
-        oracle_row(q, k, v, seg_q, seg_kv, H, S_q, S_kv, D, scale,
+        oracle_row(q, k, v, seg_q, seg_kv, H, S_q, S_kv, D, scale, causal,
                    rows[3 * r], rows[3 * r + 1], rows[3 * r + 2], s_scratch,
                    out_rows + r * D, lse_rows + r);
       free(s_scratch);
@@ -183,7 +195,8 @@ int oracle_attn_rows_f64(const uint16_t* q, const uint16_t* k, const uint16_t* v
 int oracle_attn_probs_f64(const uint16_t* q, const uint16_t* k,
                           const int32_t* seg_q, const int32_t* seg_kv,
                           double* probs,
-                          long B, long H, long S_q, long S_kv, long D, double scale) {
+                          long B, long H, long S_q, long S_kv, long D, double scale,
+                          int causal) {
   if (check_shape(B, H, S_q, S_kv, D)) return 1;
   if ((seg_q == NULL) != (seg_kv == NULL)) return 1;
   for (long b = 0; b < B; ++b)
@@ -192,10 +205,9 @@ int oracle_attn_probs_f64(const uint16_t* q, const uint16_t* k,
         const uint16_t* qi = q + ((b * H + h) * S_q + i) * D;
         const uint16_t* kb = k + (b * H + h) * S_kv * D;
         double* prow = probs + ((b * H + h) * S_q + i) * S_kv;
-        int32_t sid = seg_q ? seg_q[b * S_q + i] : 0;
         double m = -INFINITY;
         for (long j = 0; j < S_kv; ++j) {
-          int allowed = !seg_q || seg_kv[b * S_kv + j] == sid;
+          int allowed = key_allowed(seg_q, seg_kv, S_q, S_kv, b, i, j, causal);
           if (!allowed) { prow[j] = -INFINITY; continue; }
           double dot = 0.0;
           for (long d = 0; d < D; ++d)

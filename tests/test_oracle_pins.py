@@ -32,8 +32,9 @@ def f64(b):
     return wl.bf16_bits_to_f32(b).astype(np.float64)
 
 
-def brute_force(q, k, v, seg_q, seg_kv, scale):
-    """Pure-Python double loop: the full masked score matrix, then normalise."""
+def brute_force(q, k, v, seg_q, seg_kv, scale, causal=False):
+    """Pure-Python double loop: the full masked score matrix, then normalise.
+    causal: key j visible to query i only if j <= i + (S_kv - S_q)."""
     qf, kf, vf = f64(q), f64(k), f64(v)
     B, H, Sq, D = q.shape
     Skv = k.shape[2]
@@ -43,6 +44,9 @@ def brute_force(q, k, v, seg_q, seg_kv, scale):
         row = []
         for j in range(Skv):
             if seg_q is not None and seg_q[b, i] != seg_kv[b, j]:
+                row.append(None)
+                continue
+            if causal and j > i + (Skv - Sq):
                 row.append(None)
                 continue
             row.append(scale * math.fsum(qf[b, h, i, d] * kf[b, h, j, d] for d in range(D)))
@@ -93,6 +97,21 @@ def test_brute_force_tiny(shape, n_ids, seed):
     assert np.all(lse[~finite] == -np.inf)
 
 
+@pytest.mark.parametrize("shape,n_ids,seed", [
+    ((1, 2, 6, 6, 3), 0, 21), ((2, 1, 5, 8, 4), 2, 22), ((1, 1, 8, 3, 2), 0, 23),
+    ((2, 2, 7, 7, 3), 3, 24),
+])
+def test_brute_force_tiny_causal(shape, n_ids, seed):
+    c = rand_case(*shape, seed, n_ids)
+    out, lse = oracle.attn_fwd(c["q"], c["k"], c["v"], c["seg_q"], c["seg_kv"], c["scale"],
+                               causal=True)
+    ro, rl = brute_force(c["q"], c["k"], c["v"], c["seg_q"], c["seg_kv"], c["scale"], causal=True)
+    fin = np.isfinite(rl)
+    assert np.array_equal(fin, np.isfinite(lse))
+    assert np.max(np.abs(out - ro)) <= TOL
+    assert np.max(np.abs(lse[fin] - rl[fin]), initial=0) <= TOL
+
+
 # ------------------------------------------------------------ library routine
 
 @pytest.mark.parametrize("seed,n_ids", [(5, 0), (6, 2), (7, 3)])
@@ -116,6 +135,53 @@ def test_matches_torch_sdpa_fp64(seed, n_ids):
     assert np.max(np.abs(out[nonempty] - ref[nonempty])) <= 1e-12
     assert np.max(np.abs(lse[nonempty] - ref_lse[nonempty])) <= 1e-12
     assert np.all(out[~nonempty] == 0) and np.all(lse[~nonempty] == -np.inf)
+
+
+@pytest.mark.parametrize("S_q,S_kv", [(40, 40), (25, 40), (40, 25)])
+def test_causal_matches_torch_sdpa_fp64(S_q, S_kv):
+    """torch's fp64 SDPA with the bottom-right causal boolean mask."""
+    B, H, D = 2, 2, 16
+    c = rand_case(B, H, S_q, S_kv, D, 25, 2, std=2.0)
+    q, k, v = (torch.from_numpy(f64(c[n])) for n in ("q", "k", "v"))
+    i = torch.arange(S_q)[:, None]
+    j = torch.arange(S_kv)[None, :]
+    causal = j <= i + (S_kv - S_q)
+    mask = torch.from_numpy(c["seg_q"][:, None, :, None] == c["seg_kv"][:, None, None, :]) & causal
+    mask = mask.expand(B, H, S_q, S_kv)
+    nonempty = mask.any(-1).numpy()
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask,
+                                                           scale=c["scale"]).numpy()
+    logits = (q @ k.transpose(-1, -2)) * c["scale"]
+    ref_lse = torch.logsumexp(logits.masked_fill(~mask, -math.inf), dim=-1).numpy()
+    out, lse = oracle.attn_fwd(c["q"], c["k"], c["v"], c["seg_q"], c["seg_kv"], c["scale"],
+                               causal=True)
+    assert np.max(np.abs(out[nonempty] - ref[nonempty])) <= 1e-12
+    assert np.max(np.abs(lse[nonempty] - ref_lse[nonempty])) <= 1e-12
+    assert np.all(out[~nonempty] == 0) and np.all(lse[~nonempty] == -np.inf)
+
+
+def test_causal_prefix_property_and_first_row():
+    """Causal row i (S_q = S_kv) is full attention over keys 0..i alone; the
+    first row sees only key 0: out = v_0, lse = scale q_0.k_0."""
+    B, H, S, D = 1, 2, 12, 8
+    c = wl.make_random(B, H, S, S, D, 26)
+    out, lse = oracle.attn_fwd(c["q"], c["k"], c["v"], scale=c["scale"], causal=True)
+    for i in range(S):
+        sub = {x: np.ascontiguousarray(c[x][:, :, :i + 1]) for x in ("k", "v")}
+        qi = np.ascontiguousarray(c["q"][:, :, i:i + 1])
+        o2, l2 = oracle.attn_fwd(qi, sub["k"], sub["v"], scale=c["scale"])
+        assert np.max(np.abs(out[:, :, i] - o2[:, :, 0])) <= TOL
+        assert np.max(np.abs(lse[:, :, i] - l2[:, :, 0])) <= TOL
+    assert np.array_equal(out[:, :, 0], f64(c["v"])[:, :, 0])
+    s00 = c["scale"] * np.sum(f64(c["q"])[:, :, 0] * f64(c["k"])[:, :, 0], -1)
+    assert np.max(np.abs(lse[:, :, 0] - s00)) <= 1e-14
+
+
+def test_causal_with_more_queries_than_keys_has_empty_rows():
+    c = wl.make_random(1, 1, 10, 4, 4, 27)
+    out, lse = oracle.attn_fwd(c["q"], c["k"], c["v"], scale=c["scale"], causal=True)
+    assert np.all(lse[:, :, :6] == -np.inf) and np.all(out[:, :, :6] == 0)
+    assert np.all(np.isfinite(lse[:, :, 6:]))
 
 
 # ----------------------------------------------------------------- closed forms
