@@ -147,32 +147,34 @@ class ClockSampler:
 
 # -------------------------------------------------------------- reference
 
-def oracle_rows_throughput(w, inputs, n_rows, seed=0):
+def oracle_rows_throughput(w, inputs, n_rows, seed=0, causal=False):
     """Time the fp64 oracle on n_rows random rows of the workload.
     Returns (TFLOP/s counted over allowed pairs of those rows, seconds, threads)."""
     import oracle
     rng = np.random.Generator(np.random.PCG64(seed))
     rows = np.stack([rng.integers(0, w.B, n_rows), rng.integers(0, w.H, n_rows),
                      rng.integers(0, w.S_q, n_rows)], 1).astype(np.int64)
+    lim = (lambda i: i + 1 + w.S_kv - w.S_q) if causal else (lambda i: w.S_kv)
     if inputs["seg_q"] is not None:
         sq, sk = inputs["seg_q"], inputs["seg_kv"]
-        allowed = np.array([int(np.count_nonzero(sk[b] == sq[b, i])) for b, _, i in rows])
+        allowed = np.array([int(np.count_nonzero(sk[b, :max(0, lim(i))] == sq[b, i]))
+                            for b, _, i in rows])
     else:
-        allowed = np.full(n_rows, w.S_kv)
+        allowed = np.array([min(w.S_kv, max(0, lim(i))) for _, _, i in rows])
     threads = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
     oracle.attn_rows(inputs["q"], inputs["k"], inputs["v"], rows, inputs["seg_q"],
-                     inputs["seg_kv"], w.scale, nthreads=threads)
+                     inputs["seg_kv"], w.scale, nthreads=threads, causal=causal)
     dt = time.perf_counter() - t0
     flops = 4.0 * w.D * float(allowed.sum())
     return flops / dt / 1e12, dt, threads
 
 
-def cpu_baseline(w, inputs, target_s=12.0):
+def cpu_baseline(w, inputs, target_s=12.0, causal=False):
     """Oracle on a bounded sample sized to about target_s seconds of CPU work."""
-    v, dt, thr = oracle_rows_throughput(w, inputs, 64, seed=1)
+    v, dt, thr = oracle_rows_throughput(w, inputs, 64, seed=1, causal=causal)
     n = int(max(64, min(200000, 64 * target_s / max(dt, 1e-3))))
-    v, dt, thr = oracle_rows_throughput(w, inputs, n, seed=2)
+    v, dt, thr = oracle_rows_throughput(w, inputs, n, seed=2, causal=causal)
     return {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle",
             "sample": f"{n} random (b,h,i) rows of {w.name} (all their allowed keys), "
                       f"fp64 oracle, {dt:.1f} s on {thr} threads"}
@@ -229,8 +231,9 @@ def weak_scaling_value(flops_per_rank_step: float, steps: int, world: int,
     return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
 
 
-def workload_config(w):
-    return {"workload": w.name, "B": w.B, "H": w.H, "S_q": w.S_q, "S_kv": w.S_kv, "D": w.D,
+def workload_config(w, causal=False):
+    return {"workload": w.name + ("_causal" if causal else ""),
+            "B": w.B, "H": w.H, "S_q": w.S_q, "S_kv": w.S_kv, "D": w.D, "causal": causal,
             "segments": None if w.segments is None else [list(r) for r in w.segments],
             "description": w.description,
             "l2": "inputs larger than L2 (no flush)" if algorithmic_bytes(w) > 126e6
@@ -249,6 +252,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (smaller profiling cases)")
+    ap.add_argument("--causal", action="store_true",
+                    help="causal limit within segments (vidattn_fwd_ex, VIDATTN_CAUSAL)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: total oracle time budget")
@@ -296,12 +301,14 @@ def main(argv=None):
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
 
+    flags = binding.VIDATTN_CAUSAL if args.causal else 0
+
     def step():
-        st = lib.vidattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                             None if sq is None else sq.data_ptr(),
-                             None if sk is None else sk.data_ptr(),
-                             out.data_ptr(), lse.data_ptr(), w.B, w.H, w.S_q, w.S_kv, w.D,
-                             w.scale, sh)
+        st = lib.vidattn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                None if sq is None else sq.data_ptr(),
+                                None if sk is None else sk.data_ptr(),
+                                out.data_ptr(), lse.data_ptr(), w.B, w.H, w.S_q, w.S_kv, w.D,
+                                w.scale, flags, sh)
         if st != 0:
             raise RuntimeError(binding.status_string(st))
 
@@ -335,7 +342,7 @@ def main(argv=None):
     per_step = [ev[s].elapsed_time(ev[s + 1]) for s in range(args.steps)]
     total_ms = ev[0].elapsed_time(ev[-1])
     total_ms_max = rank_max(total_ms)
-    flops_step = wl.flops(w)
+    flops_step = wl.flops(w, causal=args.causal)
     value = weak_scaling_value(flops_step, args.steps, world, total_ms_max)
     ms_per_step = total_ms_max / args.steps
 
@@ -393,14 +400,14 @@ def main(argv=None):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, inputs)
+        cpu = cpu_baseline(w, inputs, causal=args.causal)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+            "dtype": "bf16", "data": "synthetic", "config": workload_config(w, args.causal),
             "pct_of_bf16_peak": 100.0 * value / (world * peaks["bf16"]),
             "ms_per_step_min": min(per_step), "ms_per_step_median": statistics.median(per_step),
             "hbm_gbs": algorithmic_bytes(w) / (kernel_ms * 1e-3) / 1e9,

@@ -98,6 +98,27 @@ VIDATTN_API int vidattn_fwd(const void* q, const void* k, const void* v,
                             int B, int H, int S_q, int S_kv, int D, float scale,
                             vidattn_stream_t stream);
 
+/* Flags of vidattn_fwd_ex. */
+#define VIDATTN_CAUSAL 1   /* key j visible to query i only if also j <= i + (S_kv - S_q) */
+
+/*
+ * vidattn_fwd_ex — vidattn_fwd with options.  flags = 0 is exactly
+ * vidattn_fwd.  flags = VIDATTN_CAUSAL adds a causal limit to the segment
+ * rule: query i sees key j iff the ids match (when given) and
+ * j <= i + (S_kv - S_q), the last query aligned with the last key (the
+ * causal "understanding" pathway that the vidax paper, §3.1, Cosmos
+ * paragraph, combines with full-attention generation in one backbone;
+ * combined with segment ids this is block-diagonal causal attention).  Key
+ * tiles past the limit are never loaded.  Rows that see no key give out = 0,
+ * lse = -inf.  Unknown flag bits return VIDATTN_ERR_BAD_SHAPE.  Other
+ * arguments, errors and ownership: as vidattn_fwd.
+ */
+VIDATTN_API int vidattn_fwd_ex(const void* q, const void* k, const void* v,
+                               const int32_t* seg_q, const int32_t* seg_kv,
+                               void* out, float* lse,
+                               int B, int H, int S_q, int S_kv, int D, float scale, int flags,
+                               vidattn_stream_t stream);
+
 /*
  * vidattn_fwd_host — the same operation on HOST buffers, for callers whose
  * data lives in host memory.  h_* are host pointers (pinned memory gives

@@ -58,7 +58,7 @@ class Guarded:
         assert not bool(torch.isnan(self.lse).any()), "some lse element was never written"
 
 
-def run_gpu(case, scale=None, check=True):
+def run_gpu(case, scale=None, check=True, causal=False):
     """case: dict of numpy inputs (q, k, v bf16 bits; seg_q, seg_kv int32 or None)."""
     q, k, v = (to_dev_bf16(case[n]) for n in ("q", "k", "v"))
     sq, sk = to_dev_i32(case.get("seg_q")), to_dev_i32(case.get("seg_kv"))
@@ -66,7 +66,8 @@ def run_gpu(case, scale=None, check=True):
     S_kv = case["k"].shape[2]
     g = Guarded(B, H, S_q, D)
     sc = case["scale"] if scale is None else scale
-    st = binding.vidattn_fwd(q, k, v, sq, sk, g.out, g.lse, B, H, S_q, S_kv, D, sc)
+    st = binding.vidattn_fwd_ex(q, k, v, sq, sk, g.out, g.lse, B, H, S_q, S_kv, D, sc,
+                                binding.VIDATTN_CAUSAL if causal else 0)
     assert st == 0, binding.status_string(st)
     torch.cuda.synchronize()
     assert binding.device_status() == 0
@@ -93,10 +94,11 @@ def compare(out_gpu, lse_gpu, out_ref, lse_ref, what=""):
     return {}
 
 
-def check_all_rows(case, scale=None, what=""):
-    out, lse = run_gpu(case, scale)
+def check_all_rows(case, scale=None, what="", causal=False):
+    out, lse = run_gpu(case, scale, causal=causal)
     ro, rl = oracle.attn_fwd(case["q"], case["k"], case["v"], case.get("seg_q"),
-                             case.get("seg_kv"), case["scale"] if scale is None else scale)
+                             case.get("seg_kv"), case["scale"] if scale is None else scale,
+                             causal=causal)
     return compare(bf16_to_f64(out), lse.double().cpu().numpy(), ro, rl, what)
 
 

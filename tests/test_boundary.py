@@ -31,7 +31,7 @@ def header_names():
 
 def test_header_declares_the_entry_points():
     names = set(header_names())
-    assert {"vidattn_fwd", "vidattn_fwd_host", "vidattn_status_string", "vidattn_device_status",
+    assert {"vidattn_fwd", "vidattn_fwd_ex", "vidattn_fwd_host", "vidattn_status_string", "vidattn_device_status",
             "vidattn_kernels_per_call", "vidattn_release", "vidattn_version",
             "vidattn_selftest_timeout"} <= names
     assert set(binding.exported_symbols()) == names
@@ -70,6 +70,13 @@ def call(lib, q=A, k=A, v=A, sq=None, sk=None, out=A, lse=A, B=1, H=2, Sq=256, S
 ])
 def test_argument_errors_return_before_any_launch(lib, kw, expect):
     assert call(lib, **kw) == expect
+
+
+def test_unknown_flag_bits_are_rejected(lib):
+    f = lib.vidattn_fwd_ex
+    assert f(A, A, A, None, None, A, A, 1, 2, 256, 256, 128, 0.1, 2, None) == BAD_SHAPE
+    assert f(A, A, A, None, None, A, A, 1, 2, 256, 256, 96, 0.1, 1, None) == BAD_D
+    assert f(A, A, A, None, None, A, A, 1, 2, 0, 256, 128, 0.1, 1, None) == OK
 
 
 def test_empty_query_is_a_no_op(lib):

@@ -214,6 +214,38 @@ def test_streams_other_than_the_current_one():
     assert torch.equal(lse, ref_lse)
 
 
+# ------------------------------------------------------------------ causal
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("S_q,S_kv", [(128, 128), (300, 300), (257, 513), (513, 257),
+                                      (1000, 1000), (100, 700)])
+def test_causal_shapes(S_q, S_kv, D):
+    c = wl.make_random(2, 2, S_q, S_kv, D, seed=S_q + 3 * S_kv + D)
+    check_all_rows(c, causal=True, what=f"causal Sq{S_q} Skv{S_kv} D{D}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_causal_with_segments(D):
+    c = runs_case(2, 2, ((500, 3), (300, 1), (77, 5)), D, 47)
+    check_all_rows(c, causal=True, what=f"causal + ids D{D}")
+    rng = np.random.Generator(np.random.PCG64(48))
+    seg = rng.integers(0, 3, (1, 640)).astype(np.int32)
+    c = wl.make_random(1, 2, 640, 640, D, 49, seg, seg.copy())
+    check_all_rows(c, causal=True, what=f"causal + random ids D{D}")
+
+
+def test_causal_full_size_480p_sampled_rows():
+    w = wl.WORKLOADS["video_480p"]
+    c = wl.make_inputs(w)
+    out, lse = run_gpu(c, causal=True)
+    rows = sample_rows(w.B, w.H, w.S_q, None, n_random=1024, n_heads_full=2)
+    ro, rl = oracle.attn_rows(c["q"], c["k"], c["v"], rows, None, None, c["scale"], causal=True)
+    b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+    idx = torch.from_numpy(((b * w.H + h) * w.S_q + i).astype(np.int64)).cuda()
+    compare(bf16_to_f64(out.reshape(-1, w.D)[idx]), lse.reshape(-1)[idx].double().cpu().numpy(),
+            ro, rl, what="causal 480p")
+
+
 # ---------------------------------------------------- the named workloads
 
 def test_workload_tiny_all_rows():

@@ -38,6 +38,8 @@ def load_library():
     p, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.vidattn_fwd.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, f32, p]
     lib.vidattn_fwd.restype = i32
+    lib.vidattn_fwd_ex.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, f32, i32, p]
+    lib.vidattn_fwd_ex.restype = i32
     lib.vidattn_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, f32, p]
     lib.vidattn_fwd_noalloc.restype = i32
     lib.vidattn_fwd_host.argtypes = [p, p, p, p, p, p, p,
@@ -99,6 +101,17 @@ def vidattn_fwd(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale, str
         int(B), int(H), int(S_q), int(S_kv), int(D), float(scale), _stream(stream))
 
 
+VIDATTN_CAUSAL = 1
+
+
+def vidattn_fwd_ex(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale, flags,
+                   stream=None) -> int:
+    """vidattn_fwd with flags (VIDATTN_CAUSAL).  Returns the status."""
+    return load_library().vidattn_fwd_ex(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv), _ptr(out), _ptr(lse),
+        int(B), int(H), int(S_q), int(S_kv), int(D), float(scale), int(flags), _stream(stream))
+
+
 def vidattn_fwd_noalloc(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale,
                         stream=None) -> int:
     """vidattn_fwd without any device allocation (fixed library scratch, with a
@@ -133,7 +146,7 @@ def kernels_per_call(seg_q, seg_kv, B, H, S_q, S_kv, D) -> int:
                                                    int(S_q), int(S_kv), int(D))
 
 
-def attention(q, k, v, seg_q=None, seg_kv=None, scale=None, stream=None):
+def attention(q, k, v, seg_q=None, seg_kv=None, scale=None, stream=None, causal=False):
     """Allocate out/lse with torch and run ``vidattn_fwd``.
     q: bf16 [B,H,S_q,D]; k, v: bf16 [B,H,S_kv,D]; seg_*: int32 [B,S] or None.
     Returns (out bf16 [B,H,S_q,D], lse fp32 [B,H,S_q]); raises on error."""
@@ -144,7 +157,8 @@ def attention(q, k, v, seg_q=None, seg_kv=None, scale=None, stream=None):
         scale = D ** -0.5
     out = torch.empty_like(q)
     lse = torch.empty((B, H, S_q), dtype=torch.float32, device=q.device)
-    st = vidattn_fwd(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale, stream)
+    st = vidattn_fwd_ex(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale,
+                        VIDATTN_CAUSAL if causal else 0, stream)
     if st != VIDATTN_OK:
         raise RuntimeError(f"vidattn_fwd failed: {status_string(st)} ({st})")
     return out, lse

@@ -61,6 +61,8 @@ struct FwdParams {
   int* err;                 // device error word (bit kErrTimeout: a wait timed out)
   int H, S_q, S_kv;
   int n_q_tiles, n_kv_tiles;
+  int causal;               // nonzero: key j visible to query i only if j <= i + causal_off
+  int causal_off;           // S_kv - S_q (the last query aligned with the last key)
   float c;                  // scale * log2(e)
   unsigned long long* trace; // VIDATTN_TRACE builds only: per-event clock64 stamps
 };
@@ -219,12 +221,31 @@ __device__ __forceinline__ float exp_tile(const float (&s)[kBN], float c, float 
   return s03.x + s03.y;
 }
 
+// Causal limit: one past the last key tile any query row of CTA `pair` can
+// see (all tiles when not causal; 0 when no row sees any key).
+__device__ __forceinline__ int causal_end(const FwdParams& p, int pair) {
+  if (!p.causal) return p.n_kv_tiles;
+  const int max_row = min(pair * 2 * kBM + 2 * kBM - 1, p.S_q - 1);
+  const int last_key = max_row + p.causal_off;
+  if (last_key < 0) return 0;
+  return min(p.n_kv_tiles, last_key / kBN + 1);
+}
+
+// Causal limit: does Q tile qi of CTA `pair` see only part of key tile j
+// (some key of the tile lies after its first row's limit)?  Then that tile
+// takes the masked path for that Q tile.
+__device__ __forceinline__ bool causal_partial(const FwdParams& p, int pair, int qi, int j) {
+  if (!p.causal) return false;
+  const int r0 = pair * 2 * kBM + qi * kBM;
+  return j * kBN + kBN - 1 > r0 + p.causal_off;
+}
+
 // The key-tile walk of CTA (b, pair) and, optionally, the id summary of one
 // of its two query tiles (qi), read from the classifier's output.  Each role
 // builds its own copy, so nothing stays live across the role branches.
 __device__ __forceinline__ KvWalk make_walk(const FwdParams& p, int b, int pair, int qi = -1,
                                             int4* q_summary = nullptr) {
-  KvWalk walk{nullptr, p.n_kv_tiles, 0, 0};
+  KvWalk walk{nullptr, causal_end(p, pair), 0, 0};
   if (p.q_sum == nullptr) {
     if (q_summary) *q_summary = make_int4(0, 0, 1, 0);
     return walk;
@@ -302,7 +323,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int b = blockIdx.z;
   const int h = blockIdx.y;
   const int bh = b * p.H + h;
-  const int m0 = blockIdx.x * 2 * kBM;
+  // 256-row query block of this CTA.  With the causal limit, later blocks see
+  // more keys: they are handed out first (the hardware starts CTAs in index
+  // order), so the longest work does not trail at the end of the launch.
+  const int pair = p.causal ? int(gridDim.x) - 1 - int(blockIdx.x) : int(blockIdx.x);
+  const int m0 = pair * 2 * kBM;
 
   const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
   auto sKV = [&](int s) { return sbase + C::kOffKV + s * C::kTileBytes; };
@@ -346,7 +371,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
 
   const bool has_seg = p.q_sum != nullptr;
-  const int n_kv = p.n_kv_tiles;
+  // key tiles visited end here (causal: past the last key any row sees)
+  const int n_kv = causal_end(p, pair);
 #ifdef VIDATTN_TRACE
   const bool trace_cta = p.trace != nullptr && blockIdx.x == gridDim.x / 2 &&
                          blockIdx.y == gridDim.y / 2 && blockIdx.z == 0;
@@ -360,8 +386,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const bool listed = has_seg && n_kv <= kMaxListedTiles;
   if (listed) {
     int4 q0, q1;
-    const KvWalk w = make_walk(p, b, blockIdx.x, 0, &q0);
-    make_walk(p, b, blockIdx.x, 1, &q1);
+    const KvWalk w = make_walk(p, b, pair, 0, &q0);
+    make_walk(p, b, pair, 1, &q1);
     const bool ragged = (p.S_kv % kBN) != 0;
     int* warp_cnt = reinterpret_cast<int*>(smem + C::kOffWarpCnt);
     for (int c0 = 0; c0 < n_kv; c0 += kFwdThreads) {
@@ -371,9 +397,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (jj < n_kv) {
         const int4 ks = __ldg(w.kv_sum + jj);
         act = !(ks.y < w.qmin || ks.x > w.qmax);
-        const bool last_ragged = ragged && jj == n_kv - 1;
-        const bool m0 = last_ragged || !(q0.z && ks.z && q0.x == ks.x);
-        const bool m1 = last_ragged || !(q1.z && ks.z && q1.x == ks.x);
+        const bool last_ragged = ragged && jj == p.n_kv_tiles - 1;
+        const bool m0 = last_ragged || !(q0.z && ks.z && q0.x == ks.x) ||
+                        causal_partial(p, pair, 0, jj);
+        const bool m1 = last_ragged || !(q1.z && ks.z && q1.x == ks.x) ||
+                        causal_partial(p, pair, 1, jj);
         entry = jj | (m0 ? (1 << 30) : 0) | (m1 ? int(1u << 31) : 0);
       }
       const unsigned ballot = __ballot_sync(0xffffffffu, act);
@@ -407,7 +435,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   if (warp == 9) {
     // ------------------------------------------------------------ TMA loads
     {  // the whole warp runs the loop; one elected lane issues
-      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, blockIdx.x)};
+      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, pair)};
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
@@ -460,7 +488,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // Order per tile t: S0 = Q0 K_{t+1}^T once S0_t is read, O0 += P0 V_t,
       // S1 = Q1 K_{t+1}^T once S1_t is read, O1 += P1 V_t.  K_t is load 2t
       // and V_t load 2t+1 of the ring.
-      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, blockIdx.x)};
+      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, pair)};
       int j = sched.tile(0, -1);
       if (j < n_kv) {
         auto stage = [&](int idx) { return idx % C::kStages; };
@@ -533,7 +561,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         warp_wait_phase(drain_bar, 0, &never, p.err);
       }
     } else {
-      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, blockIdx.x)};
+      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, pair)};
       int j = sched.tile(0, -1);
       if (j < n_kv) {
         int n = 0;   // K/V tiles consumed
@@ -626,7 +654,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tP = tmem + lane_off + C::kTmemP + C::kPStride * qi;
     int4 my_qs;
     const KvSched sched{listed ? tile_list : nullptr, n_list,
-                        make_walk(p, b, blockIdx.x, qi, &my_qs)};
+                        make_walk(p, b, pair, qi, &my_qs)};
     const float c = p.c;
     const bool ragged_kv = (p.S_kv % kBN) != 0;
 
@@ -639,7 +667,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (listed) {
         masked = (tile_list[t] >> (30 + qi)) & 1;
       } else {
-        masked = ragged_kv && j == n_kv - 1;
+        masked = (ragged_kv && j == p.n_kv_tiles - 1) || causal_partial(p, pair, qi, j);
         if (has_seg) {
           const int4 ks = __ldg(sched.walk.kv_sum + j);
           masked = masked || !(my_qs.z && ks.z && my_qs.x == ks.x);
@@ -677,7 +705,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             float mx = -INFINITY;
 #pragma unroll
             for (int x = 0; x < kBN; ++x) {
-              bool valid = (j0 + x) < p.S_kv;
+              bool valid = (j0 + x) < p.S_kv && (!p.causal || j0 + x <= row + p.causal_off);
               if (has_seg && valid) valid = __ldg(seg_kv_b + j0 + x) == my_seg;
               s[x] = valid ? s[x] * c : -INFINITY;
               mx = fmaxf(mx, s[x]);
@@ -763,7 +791,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           rs = 0.f;
           const int j0 = j * kBN;
           auto allowed = [&](int x) {
-            bool valid = (j0 + x) < p.S_kv;
+            bool valid = (j0 + x) < p.S_kv && (!p.causal || j0 + x <= row + p.causal_off);
             if (has_seg && valid) valid = __ldg(seg_kv_b + j0 + x) == my_seg;
             return valid;
           };

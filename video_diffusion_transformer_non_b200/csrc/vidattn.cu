@@ -262,7 +262,8 @@ int check_args(const void* q, const void* k, const void* v, const int32_t* seg_q
 template <int D>
 int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32_t* seg_q,
                const int32_t* seg_kv, const int4* q_sum, const int4* kv_sum, void* out,
-               float* lse, int B, int H, int S_q, int S_kv, float scale, cudaStream_t stream) {
+               float* lse, int B, int H, int S_q, int S_kv, float scale, cudaStream_t stream,
+               int flags = 0) {
   CUtensorMap tq, tk, tv;
   const int64_t BH = int64_t(B) * H;
   // With no keys the K/V maps are never read; they are encoded over q.
@@ -284,6 +285,8 @@ int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32
   p.S_kv = S_kv;
   p.n_q_tiles = (S_q + kBM - 1) / kBM;
   p.n_kv_tiles = (S_kv + kBN - 1) / kBN;
+  p.causal = (flags & VIDATTN_CAUSAL) ? 1 : 0;
+  p.causal_off = S_kv - S_q;
   p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
 #ifdef VIDATTN_TRACE
   p.trace = g_trace;
@@ -348,6 +351,14 @@ VIDATTN_API int vidattn_kernels_per_call(const int32_t* seg_q, const int32_t* se
 VIDATTN_API int vidattn_fwd(const void* q, const void* k, const void* v, const int32_t* seg_q,
                             const int32_t* seg_kv, void* out, float* lse, int B, int H, int S_q,
                             int S_kv, int D, float scale, vidattn_stream_t stream_) {
+  return vidattn_fwd_ex(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale, 0, stream_);
+}
+
+VIDATTN_API int vidattn_fwd_ex(const void* q, const void* k, const void* v,
+                               const int32_t* seg_q, const int32_t* seg_kv, void* out, float* lse,
+                               int B, int H, int S_q, int S_kv, int D, float scale, int flags,
+                               vidattn_stream_t stream_) {
+  if (flags & ~VIDATTN_CAUSAL) return VIDATTN_ERR_BAD_SHAPE;
   int st = check_args(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D);
   if (st != VIDATTN_OK) return st;
   if (!std::isfinite(scale)) return VIDATTN_ERR_BAD_SHAPE;
@@ -374,9 +385,9 @@ VIDATTN_API int vidattn_fwd(const void* q, const void* k, const void* v, const i
   }
   if (D == 64)
     return launch_fwd<64>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
-                          stream);
+                          stream, flags);
   return launch_fwd<128>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
-                         stream);
+                         stream, flags);
 }
 
 VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h_v,

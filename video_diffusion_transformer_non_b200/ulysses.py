@@ -1,0 +1,114 @@
+"""Sequence-parallel attention across GPUs (DeepSpeed-Ulysses layout).
+
+The vidax paper (§2, "Spatiotemporal tensor and sequence sharding") shards
+video tokens across devices between attention layers and, for attention only,
+transposes to a head-sharded view with all_to_all and back; CogVideoX1.5's
+~45k-token joint sequence needs four such devices (§4 and Table 2).  Here:
+
+* every rank holds q, k, v for its contiguous 1/P of the sequence and all H
+  heads, bf16 [B, H, S/P, D], and its slice of the segment ids, int32 [B, S/P];
+* one all_to_all per tensor gives each rank all S tokens of H/P heads
+  (rank r gets heads [r H/P, (r+1) H/P)), the ids are all_gathered;
+* the attention runs on that head shard through the library's C ABI
+  (``vidattn_fwd_ex``), every key of the full sequence visible to every query;
+* one all_to_all returns out [B, H, S/P, D] and lse [B, H, S/P] to the
+  sequence-sharded layout.
+
+With ``n_chunks > 1`` the heads of the shard are processed in chunks so the
+exchange of one chunk overlaps the attention of the previous one (NCCL runs
+the collectives on its own stream).  The collective is torch.distributed's
+(NCCL over NVLink on GPUs, gloo on CPU for the tests); the data-path kernel is
+vidattn's.  `attn_fn` replaces the attention call (tests on CPU).
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import binding
+
+
+def _world(group):
+    return dist.get_world_size(group) if dist.is_initialized() else 1
+
+
+class _Exchange:
+    """One all_to_all in flight and the reshaping that follows it."""
+
+    def __init__(self, send, finish, P, group):
+        self.recv = torch.empty_like(send)
+        self.finish = finish
+        self.work = dist.all_to_all_single(self.recv, send, group=group, async_op=True) \
+            if P > 1 else None
+        if P == 1:
+            self.recv = send
+
+    def result(self):
+        if self.work is not None:
+            self.work.wait()
+        return self.finish(self.recv)
+
+
+def _seq_to_heads(x: torch.Tensor, P: int, group) -> _Exchange:
+    """[B, H, Sl, *r] sequence shard -> [B, H/P, P*Sl, *r] head shard."""
+    B, H, Sl = x.shape[:3]
+    rest = x.shape[3:]
+    send = x.reshape(B, P, H // P, Sl, *rest).movedim(1, 0).contiguous()
+    # recv[p] = this rank's heads from sequence shard p
+    return _Exchange(send, lambda r: r.movedim(0, 2).reshape(B, H // P, P * Sl, *rest)
+                     .contiguous(), P, group)
+
+
+def _heads_to_seq(y: torch.Tensor, P: int, group) -> _Exchange:
+    """[B, H/P, S, *r] head shard -> [B, H, S/P, *r] sequence shard."""
+    B, Hl, S = y.shape[:3]
+    rest = y.shape[3:]
+    Sl = S // P
+    send = y.reshape(B, Hl, P, Sl, *rest).movedim(2, 0).contiguous()
+    # recv[p] = this rank's sequence shard for head group p
+    return _Exchange(send, lambda r: r.movedim(0, 1).reshape(B, P * Hl, Sl, *rest)
+                     .contiguous(), P, group)
+
+
+def _cuda_attention(q, k, v, seg_q, seg_kv, scale, causal):
+    return binding.attention(q, k, v, seg_q, seg_kv, scale, causal=causal)
+
+
+def ulysses_attention(q, k, v, seg=None, scale=None, causal=False, group=None, n_chunks=1,
+                      attn_fn=None):
+    """Attention over a sequence sharded across the ranks of `group`.
+
+    q, k, v: [B, H, S/P, D] (this rank's contiguous sequence shard; H divisible
+    by P * n_chunks); seg: int32 [B, S/P] or None.  Returns (out [B, H, S/P, D],
+    lse fp32 [B, H, S/P]) for this rank's shard, equal to the corresponding
+    rows of single-device attention over the whole sequence.  Head chunk c's
+    attention starts once its own inputs have arrived, while later chunks'
+    exchanges are still in flight."""
+    P = _world(group)
+    B, H, Sl, D = q.shape
+    if H % (P * n_chunks):
+        raise ValueError(f"H={H} must be divisible by world size {P} x chunks {n_chunks}")
+    if scale is None:
+        scale = D ** -0.5
+    attn = attn_fn or _cuda_attention
+    seg_full = None
+    if seg is not None:
+        if P == 1:
+            seg_full = seg.contiguous()
+        else:
+            parts = [torch.empty_like(seg) for _ in range(P)]
+            dist.all_gather(parts, seg.contiguous(), group=group)
+            seg_full = torch.cat(parts, dim=1).contiguous()
+    Hc = H // n_chunks
+    inputs = []
+    for c in range(n_chunks):          # every input exchange goes out first
+        hs = slice(c * Hc, (c + 1) * Hc)
+        inputs.append([_seq_to_heads(t[:, hs], P, group) for t in (q, k, v)])
+    outputs = []
+    for c in range(n_chunks):
+        qh, kh, vh = (x.result() for x in inputs[c])
+        o, l = attn(qh, kh, vh, seg_full, seg_full, scale, causal)
+        outputs.append((_heads_to_seq(o, P, group), _heads_to_seq(l, P, group)))
+    outs = [o.result() for o, _ in outputs]
+    lses = [l.result() for _, l in outputs]
+    return torch.cat(outs, dim=1), torch.cat(lses, dim=1)

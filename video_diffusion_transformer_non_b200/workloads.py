@@ -170,6 +170,17 @@ def allowed_pairs(w_or_seg_q, seg_kv=None, S_q=None, S_kv=None, B=None) -> int:
     return int(total)
 
 
-def flops(w: Workload) -> float:
+def causal_pairs(w: Workload) -> int:
+    """Allowed pairs under the causal limit (key j <= query i, S_q = S_kv) and
+    segment equality: n (n + 1) / 2 per id holding n tokens, per sample."""
+    if w.segments is None:
+        return w.B * w.S_q * (w.S_q + 1) // 2
+    per_id = {}
+    for n, sid in w.segments:
+        per_id[sid] = per_id.get(sid, 0) + n
+    return w.B * sum(n * (n + 1) // 2 for n in per_id.values())
+
+
+def flops(w: Workload, causal: bool = False) -> float:
     """4*D flops per allowed (query, key) pair per head: QK^T and PV."""
-    return 4.0 * w.H * w.D * allowed_pairs(w)
+    return 4.0 * w.H * w.D * (causal_pairs(w) if causal else allowed_pairs(w))
