@@ -231,8 +231,13 @@ def weak_scaling_value(flops_per_rank_step: float, steps: int, world: int,
     return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
 
 
-def workload_config(w, causal=False):
-    return {"workload": w.name + ("_causal" if causal else ""),
+def rope_algorithmic_bytes(w) -> int:
+    """q and k read once and written once, bf16."""
+    return 2 * 2 * 2 * w.B * w.H * w.S_q * w.D
+
+
+def workload_config(w, causal=False, rope=False):
+    return {"workload": w.name + ("_causal" if causal else "") + ("_rope" if rope else ""),
             "B": w.B, "H": w.H, "S_q": w.S_q, "S_kv": w.S_kv, "D": w.D, "causal": causal,
             "segments": None if w.segments is None else [list(r) for r in w.segments],
             "description": w.description,
@@ -258,6 +263,11 @@ def main(argv=None):
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: total oracle time budget")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--rope", action="store_true",
+                    help="each step rotates q and k (vidattn_rope3d, the workload's 3D RoPE "
+                         "convention) before the attention")
+    ap.add_argument("--rope-half-split", action="store_true",
+                    help="with --rope: pair features k and k + d/2 instead of 2k and 2k+1")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -302,9 +312,32 @@ def main(argv=None):
     sh = stream.cuda_stream
 
     flags = binding.VIDATTN_CAUSAL if args.causal else 0
+    use_rope = args.rope
+    rope_interleaved = w.rope_interleaved and not args.rope_half_split
+    # the attention reads the rotated q and k when the step includes the rotation
+    qa, ka = (torch.empty_like(q), torch.empty_like(k)) if use_rope else (q, k)
+    rope_ev = []     # (start, end) event pairs around each timed rotation launch
 
-    def step():
-        st = lib.vidattn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+    def rope_launch():
+        T, Hg, Wg = w.rope_grid
+        d_t, d_h, d_w = w.rope_bands
+        st = lib.vidattn_rope3d(q.data_ptr(), k.data_ptr(), qa.data_ptr(), ka.data_ptr(),
+                                w.B, w.H, w.S_q, w.D, *q.stride()[:3], T, Hg, Wg, w.rope_offset,
+                                d_t, d_h, d_w, w.rope_theta,
+                                0 if rope_interleaved else binding.VIDATTN_ROPE_HALF_SPLIT, sh)
+        if st != 0:
+            raise RuntimeError(binding.status_string(st))
+
+    def step(timed=False):
+        if use_rope:
+            if timed:
+                e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                e[0].record(stream)
+            rope_launch()
+            if timed:
+                e[1].record(stream)
+                rope_ev.append(e)
+        st = lib.vidattn_fwd_ex(qa.data_ptr(), ka.data_ptr(), v.data_ptr(),
                                 None if sq is None else sq.data_ptr(),
                                 None if sk is None else sk.data_ptr(),
                                 out.data_ptr(), lse.data_ptr(), w.B, w.H, w.S_q, w.S_kv, w.D,
@@ -332,7 +365,7 @@ def main(argv=None):
     torch.cuda.synchronize(dev)
     ev[0].record(stream)
     for s in range(args.steps):
-        step()
+        step(timed=True)
         ev[s + 1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -340,6 +373,7 @@ def main(argv=None):
     if binding.device_status() != 0:
         raise RuntimeError("device error during the timed region")
     per_step = [ev[s].elapsed_time(ev[s + 1]) for s in range(args.steps)]
+    rope_ms = [a.elapsed_time(b) for a, b in rope_ev]
     total_ms = ev[0].elapsed_time(ev[-1])
     total_ms_max = rank_max(total_ms)
     flops_step = wl.flops(w, causal=args.causal)
@@ -358,7 +392,20 @@ def main(argv=None):
         hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
         ptr = lambda t: None if t is None else t.data_ptr()
 
+        def e2e_step_rope():
+            q.copy_(hq.view(torch.bfloat16), non_blocking=True)
+            k.copy_(hk.view(torch.bfloat16), non_blocking=True)
+            v.copy_(hv.view(torch.bfloat16), non_blocking=True)
+            if hsq is not None:
+                sq.copy_(hsq, non_blocking=True)
+                sk.copy_(hsk, non_blocking=True)
+            step()
+            hout.copy_(out.view(torch.int16), non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
         def e2e_step():
+            if use_rope:
+                return e2e_step_rope()
             st = lib.vidattn_fwd_host(ptr(hq), ptr(hk), ptr(hv), ptr(hsq), ptr(hsk), ptr(hout),
                                       ptr(hlse), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                       ptr(sq), ptr(sk), out.data_ptr(), lse.data_ptr(),
@@ -387,7 +434,8 @@ def main(argv=None):
                "steps": n_e2e, "ms_per_step": e_ms / n_e2e}
 
     peaks = load_peaks()
-    kernel_ms = statistics.mean(per_step)   # one attention launch (+ classify) per step
+    # one attention launch (+ classify) per step, after the rotation when there is one
+    kernel_ms = statistics.mean(per_step) - (statistics.mean(rope_ms) if rope_ms else 0.0)
     achieved = flops_step / (kernel_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": UNIT,
                 "frac": achieved / peaks["bf16"],
@@ -398,6 +446,22 @@ def main(argv=None):
                 "algorithmic_flops_per_launch": flops_step,
                 "algorithmic_bytes_per_launch": algorithmic_bytes(w)}
 
+    rope = None
+    if use_rope:
+        r_ms = statistics.mean(rope_ms)
+        r_bytes = rope_algorithmic_bytes(w)
+        r_gbs = r_bytes / (r_ms * 1e-3) / 1e9
+        rope = {"kernel": f"rope3d_kernel<{w.D}, {'interleaved' if rope_interleaved else 'half-split'}>",
+                "ms_per_launch": r_ms, "ms_per_launch_min": min(rope_ms),
+                "share_of_step": r_ms / statistics.mean(per_step),
+                "convention": {"grid": list(w.rope_grid), "offset": w.rope_offset,
+                               "bands": list(w.rope_bands), "theta": w.rope_theta,
+                               "pairing": "interleaved" if rope_interleaved else "half-split"},
+                "roofline": {"bound": "hbm", "achieved": r_gbs, "peak": peaks["hbm"],
+                             "unit": "GB/s", "frac": r_gbs / peaks["hbm"],
+                             "traffic": None, "peak_source": f"{peaks['source']} HBM copy",
+                             "algorithmic_bytes_per_launch": r_bytes}}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, inputs, causal=args.causal)
@@ -407,13 +471,15 @@ def main(argv=None):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic", "config": workload_config(w, args.causal),
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, args.causal, rope=use_rope),
             "pct_of_bf16_peak": 100.0 * value / (world * peaks["bf16"]),
             "ms_per_step_min": min(per_step), "ms_per_step_median": statistics.median(per_step),
             "hbm_gbs": algorithmic_bytes(w) / (kernel_ms * 1e-3) / 1e9,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps * binding.kernels_per_call(
-                sq, sk, w.B, w.H, w.S_q, w.S_kv, w.D),
+            "gpu_launches": args.steps * (binding.kernels_per_call(
+                sq, sk, w.B, w.H, w.S_q, w.S_kv, w.D) + (1 if use_rope else 0)),
+            "rope3d": rope,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -170,6 +170,61 @@ VIDATTN_API int vidattn_fwd_noalloc(const void* q, const void* k, const void* v,
                                     int B, int H, int S_q, int S_kv, int D, float scale,
                                     vidattn_stream_t stream);
 
+#define VIDATTN_ROPE_HALF_SPLIT 1   /* pair feature k with k + d/2 instead of 2k with 2k+1 */
+
+/*
+ * vidattn_rope3d — 3D rotary position embedding of q and k, the step right
+ * before the attention in the video DiT families.  The vidax paper (§2,
+ * "3D RoPE, 3D VAEs, and flash attention") rotates q and k over the time,
+ * height and width axes of the video latent, keeps each family's own
+ * convention (the conventions do not interchange), and prints no formula.
+ * This entry point applies the rotary embedding of RoFormer (Su et al.,
+ * 2021) per axis:
+ *
+ *   the D features of a head are cut into three contiguous bands of
+ *   d_t, d_h and d_w features (in that order; each even, d_t+d_h+d_w = D; a
+ *   band may be empty).  Video token n (0 <= n < T*Hg*Wg) sits at sequence
+ *   index token_offset + n and has coordinates t = n / (Hg*Wg),
+ *   h = (n / Wg) % Hg, w = n % Wg.  In a band of d features, pair k
+ *   (0 <= k < d/2) is the features (2k, 2k+1) of the band, or (k, k + d/2)
+ *   with VIDATTN_ROPE_HALF_SPLIT, and is turned by
+ *   a = coord * theta^(-2k/d), coord being the token's coordinate on the
+ *   band's axis:  (x, y) -> (x cos a - y sin a, x sin a + y cos a).
+ *   Every other token (text, padding) is copied unchanged.
+ *
+ *   q_in, k_in   bf16, logical shape [B,H,S,D], element (b,h,s,f) at
+ *                in + b*stride_b + h*stride_h + s*stride_s + f (features
+ *                contiguous), device, 16-byte aligned; strides in elements,
+ *                multiples of 8.  [B,H,S,D] contiguous is (H*S*D, S*D, D);
+ *                the [B,S,H,D] output of a q/k projection is (S*H*D, D, H*D).
+ *   q_out, k_out bf16 [B,H,S,D] contiguous, device, 16-byte aligned, written.
+ *                Either the input itself (in place, contiguous input only)
+ *                or a buffer that does not overlap it.
+ *   k_in, k_out  both NULL to rotate q only.
+ *   B, H >= 1, 2*B*H < 2^31;  D = 64 or 128.
+ *   T, Hg, Wg >= 1; token_offset >= 0; token_offset + T*Hg*Wg <= S.
+ *   theta        finite, > 0 (10000 in the common conventions).
+ *   flags        0 or VIDATTN_ROPE_HALF_SPLIT.
+ *   stream       enqueued, not synchronised.
+ *
+ * Arithmetic: angles in fp64 reduced to [-pi, pi], sine and cosine in fp32,
+ * the rotation in fp32 from the bf16 inputs, the result rounded once to bf16
+ * (nearest even).  Tokens outside the video range and coordinate 0 reproduce
+ * the input bit for bit.
+ *
+ * Errors: argument errors return their status before anything is enqueued
+ * (NULL for q_in/q_out, or for exactly one of k_in/k_out; UNSUPPORTED_D;
+ * MISALIGNED for a pointer or a stride; BAD_SHAPE for the rest, unknown flag
+ * bits included); VIDATTN_ERR_CUDA if the launch fails.  One kernel, no
+ * allocation.
+ */
+VIDATTN_API int vidattn_rope3d(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                               int B, int H, int S, int D,
+                               long long stride_b, long long stride_h, long long stride_s,
+                               int T, int Hg, int Wg, int token_offset,
+                               int d_t, int d_h, int d_w, double theta, int flags,
+                               vidattn_stream_t stream);
+
 /* A static, human-readable name for a status code. */
 VIDATTN_API const char* vidattn_status_string(int status);
 

@@ -31,11 +31,22 @@ def _bf16_to_f64(bits: np.ndarray) -> np.ndarray:
 
 
 def rope3d_f64(x_bits: np.ndarray, grid, bands, theta: float = 10000.0,
-               interleaved: bool = True, token_offset: int = 0) -> np.ndarray:
+               interleaved: bool = True, token_offset: int = 0, S: int | None = None,
+               rows=None) -> np.ndarray:
     """x_bits: uint16 bf16 bits [B, H, S, D].  grid = (T, Hg, Wg);
-    bands = (d_t, d_h, d_w).  Returns float64 [B, H, S, D]."""
+    bands = (d_t, d_h, d_w).  Returns float64 [B, H, S, D].
+
+    With ``rows`` (sequence indices, ascending) x_bits holds only those tokens,
+    [B, H, len(rows), D], of a sequence of ``S`` tokens; the result is the
+    same rows of the full result."""
     x = _bf16_to_f64(x_bits)
-    B, H, S, D = x.shape
+    B, H, n_rows, D = x.shape
+    if rows is None:
+        rows = np.arange(n_rows)
+        S = n_rows
+    rows = np.asarray(rows, dtype=np.int64)
+    if rows.shape != (n_rows,) or S is None:
+        raise ValueError("rows must name one sequence index per token, with S given")
     T, Hg, Wg = grid
     if sum(bands) != D or any(d % 2 for d in bands):
         raise ValueError("bands must be even and sum to D")
@@ -43,15 +54,16 @@ def rope3d_f64(x_bits: np.ndarray, grid, bands, theta: float = 10000.0,
     if token_offset < 0 or token_offset + n_video > S:
         raise ValueError("video tokens must lie inside the sequence")
     out = x.copy()
-    n = np.arange(n_video)
+    inside = (rows >= token_offset) & (rows < token_offset + n_video)
+    n = rows[inside] - token_offset
     coords = (n // (Hg * Wg), (n // Wg) % Hg, n % Wg)
-    tok = slice(token_offset, token_offset + n_video)
+    tok = np.nonzero(inside)[0]
     start = 0
     for d, coord in zip(bands, coords):
         half = d // 2
         k = np.arange(half)
         freq = theta ** (-2.0 * k / d)                    # [half]
-        angle = coord[:, None].astype(np.float64) * freq[None, :]   # [n_video, half]
+        angle = coord[:, None].astype(np.float64) * freq[None, :]   # [tokens, half]
         c, s = np.cos(angle), np.sin(angle)
         if interleaved:
             i0 = start + 2 * k
@@ -59,9 +71,9 @@ def rope3d_f64(x_bits: np.ndarray, grid, bands, theta: float = 10000.0,
         else:
             i0 = start + k
             i1 = i0 + half
-        xa = x[:, :, tok, i0]
-        xb = x[:, :, tok, i1]
-        out[:, :, tok, i0] = xa * c - xb * s
-        out[:, :, tok, i1] = xa * s + xb * c
+        xa = x[:, :, tok][..., i0]
+        xb = x[:, :, tok][..., i1]
+        out[:, :, tok[:, None], i0[None, :]] = xa * c - xb * s
+        out[:, :, tok[:, None], i1[None, :]] = xa * s + xb * c
         start += d
     return out

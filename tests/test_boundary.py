@@ -133,3 +133,34 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "library_path", lambda: str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         binding.load_library()
+
+
+def rope(lib, q=A, k=A, qo=A + 0x100000, ko=A + 0x200000, B=1, H=2, S=128, D=128,
+         sb=2 * 128 * 128, sh=128 * 128, ss=128, T=2, Hg=4, Wg=8, off=0, bands=(44, 42, 42),
+         theta=10000.0, flags=0):
+    return lib.vidattn_rope3d(q, k, qo, ko, B, H, S, D, sb, sh, ss, T, Hg, Wg, off, *bands,
+                              theta, flags, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), NULL), (dict(qo=None), NULL), (dict(k=None), NULL), (dict(ko=None), NULL),
+    (dict(D=96, bands=(32, 32, 32)), BAD_D),
+    (dict(flags=2), BAD_SHAPE), (dict(B=0), BAD_SHAPE), (dict(H=0), BAD_SHAPE),
+    (dict(S=0), BAD_SHAPE), (dict(S=63), BAD_SHAPE), (dict(off=65), BAD_SHAPE),
+    (dict(off=-1, S=200), BAD_SHAPE), (dict(T=0), BAD_SHAPE), (dict(Wg=-8), BAD_SHAPE),
+    (dict(bands=(43, 43, 42)), BAD_SHAPE), (dict(bands=(44, 42, 40)), BAD_SHAPE),
+    (dict(bands=(-2, 66, 64)), BAD_SHAPE),
+    (dict(theta=0.0), BAD_SHAPE), (dict(theta=-1.0), BAD_SHAPE),
+    (dict(theta=float("inf")), BAD_SHAPE), (dict(theta=float("nan")), BAD_SHAPE),
+    (dict(B=40000, H=40000), BAD_SHAPE),
+    (dict(q=A + 8), MISALIGNED), (dict(ko=A + 2), MISALIGNED),
+    (dict(ss=132), MISALIGNED), (dict(sh=4), MISALIGNED), (dict(sb=12), MISALIGNED),
+])
+def test_rope3d_argument_errors_return_before_any_launch(lib, kw, expect):
+    assert rope(lib, **kw) == expect
+
+
+def test_rope3d_q_only_is_accepted_by_the_checks(lib):
+    """k_in and k_out both NULL passes the argument checks (then needs a GPU)."""
+    st = rope(lib, k=None, ko=None)
+    assert st in (OK, CUDA, NO_DEVICE)

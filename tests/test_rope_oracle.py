@@ -80,6 +80,16 @@ def test_band_of_one_axis_sees_only_that_coordinate():
     assert np.array_equal(y[9, 8:], y[0, 8:]) and not np.allclose(y[9, :8], y[0, :8])
 
 
+def test_row_subset_matches_full_result():
+    """Rows computed on their own equal the same rows of the whole sequence."""
+    grid, bands = (3, 4, 5), (16, 24, 24)
+    x = _rand_bits((2, 2, 75, 64), 6)
+    full = rope3d_f64(x, grid, bands, token_offset=9, interleaved=False)
+    rows = np.array([0, 8, 9, 10, 33, 68, 69, 74])
+    part = rope3d_f64(x[:, :, rows], grid, bands, token_offset=9, interleaved=False, S=75, rows=rows)
+    assert np.array_equal(part, full[:, :, rows])
+
+
 def test_pairings_differ():
     """The two pairings are different rotations (the conventions are not
     interchangeable)."""
@@ -127,15 +137,17 @@ import inspect
 import oracle.rope3d as _rope_mod
 
 ROPE_MUTATIONS = {
-    "rotation_sign": ("out[:, :, tok, i0] = xa * c - xb * s", "out[:, :, tok, i0] = xa * c + xb * s"),
-    "rotation_direction": ("out[:, :, tok, i1] = xa * s + xb * c", "out[:, :, tok, i1] = -xa * s + xb * c"),
+    "rotation_sign": ("i0[None, :]] = xa * c - xb * s", "i0[None, :]] = xa * c + xb * s"),
+    "rotation_direction": ("i1[None, :]] = xa * s + xb * c", "i1[None, :]] = -xa * s + xb * c"),
     "freq_exponent": ("freq = theta ** (-2.0 * k / d)", "freq = theta ** (-1.0 * k / d)"),
     "freq_over_D": ("freq = theta ** (-2.0 * k / d)", "freq = theta ** (-2.0 * k / D)"),
     "hw_swapped": ("coords = (n // (Hg * Wg), (n // Wg) % Hg, n % Wg)",
                    "coords = (n // (Hg * Wg), n % Wg, (n // Wg) % Hg)"),
     "w_mod_Hg": ("coords = (n // (Hg * Wg), (n // Wg) % Hg, n % Wg)",
                  "coords = (n // (Hg * Wg), (n // Wg) % Hg, n % Hg)"),
-    "offset_ignored": ("tok = slice(token_offset, token_offset + n_video)", "tok = slice(0, n_video)"),
+    "offset_not_subtracted": ("n = rows[inside] - token_offset", "n = rows[inside]"),
+    "range_ignores_offset": ("inside = (rows >= token_offset) & (rows < token_offset + n_video)",
+                             "inside = rows < n_video"),
     "pairing_swapped": ("if interleaved:", "if not interleaved:"),
     "half_split_stride": ("i1 = i0 + half", "i1 = i0 + 1"),
     "band_start_not_advanced": ("start += d", "start += 0"),

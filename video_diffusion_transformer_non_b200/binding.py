@@ -56,6 +56,10 @@ def load_library():
     lib.vidattn_kernels_per_call.restype = i32
     lib.vidattn_selftest_timeout.argtypes = [i32, p]
     lib.vidattn_selftest_timeout.restype = i32
+    i64, f64 = ctypes.c_longlong, ctypes.c_double
+    lib.vidattn_rope3d.argtypes = [p, p, p, p, i32, i32, i32, i32, i64, i64, i64,
+                                   i32, i32, i32, i32, i32, i32, i32, f64, i32, p]
+    lib.vidattn_rope3d.restype = i32
     lib.vidattn_version.argtypes = []
     lib.vidattn_version.restype = ctypes.c_char_p
     _lib = lib
@@ -162,3 +166,47 @@ def attention(q, k, v, seg_q=None, seg_kv=None, scale=None, stream=None, causal=
     if st != VIDATTN_OK:
         raise RuntimeError(f"vidattn_fwd failed: {status_string(st)} ({st})")
     return out, lse
+
+
+VIDATTN_ROPE_HALF_SPLIT = 1
+
+
+def vidattn_rope3d(q_in, k_in, q_out, k_out, B, H, S, D, stride_b, stride_h, stride_s,
+                   T, Hg, Wg, token_offset, d_t, d_h, d_w, theta, flags, stream=None) -> int:
+    """Enqueue the 3D rotary embedding of q (and k) on ``stream``.  Returns the status."""
+    return load_library().vidattn_rope3d(
+        _ptr(q_in), _ptr(k_in), _ptr(q_out), _ptr(k_out), int(B), int(H), int(S), int(D),
+        int(stride_b), int(stride_h), int(stride_s), int(T), int(Hg), int(Wg), int(token_offset),
+        int(d_t), int(d_h), int(d_w), float(theta), int(flags), _stream(stream))
+
+
+def rope3d(q, k=None, grid=None, bands=None, theta=10000.0, interleaved=True, token_offset=0,
+           out_q=None, out_k=None, stream=None):
+    """Rotate q (and k) by the 3D rotary embedding; returns (q_rot, k_rot or None),
+    bf16 [B,H,S,D] contiguous.  q, k: bf16 [B,H,S,D] tensors whose last dim is
+    contiguous, any other strides (a [B,S,H,D] tensor's ``transpose(1, 2)`` view
+    works); grid = (T, Hg, Wg) of the video tokens; bands = (d_t, d_h, d_w).
+    ``out_q=q`` (and ``out_k=k``) rotates a contiguous input in place."""
+    import torch
+    B, H, S, D = q.shape
+    if k is not None and k.shape != q.shape:
+        raise ValueError("q and k must have the same shape")
+    if k is not None and k.stride() != q.stride():
+        raise ValueError("q and k must have the same strides")
+    if q.stride(3) != 1:
+        raise ValueError("the feature dim must be contiguous")
+    out_q = torch.empty((B, H, S, D), dtype=q.dtype, device=q.device) if out_q is None else out_q
+    if k is not None and out_k is None:
+        out_k = torch.empty((B, H, S, D), dtype=k.dtype, device=k.device)
+    for o in (out_q, out_k):
+        if o is not None and (tuple(o.shape) != (B, H, S, D) or not o.is_contiguous()):
+            raise ValueError("outputs must be contiguous [B,H,S,D]")
+    T, Hg, Wg = grid
+    d_t, d_h, d_w = bands
+    sb, sh, ss, _ = q.stride()
+    st = vidattn_rope3d(q, k, out_q, out_k if k is not None else None, B, H, S, D, sb, sh, ss,
+                        T, Hg, Wg, token_offset, d_t, d_h, d_w, theta,
+                        0 if interleaved else VIDATTN_ROPE_HALF_SPLIT, stream)
+    if st != VIDATTN_OK:
+        raise RuntimeError(f"vidattn_rope3d failed: {status_string(st)} ({st})")
+    return out_q, out_k

@@ -21,7 +21,7 @@ OUT = os.path.join(CSRC, "libvidattn.so")
 PROBES_OUT = os.path.join(CSRC, "libvidattn_probes.so")
 # (output, sources, dependencies)
 TARGETS = [
-    (OUT, ["vidattn.cu"], ["vidattn.cu", "fwd_kernel.cuh", "classify.cuh", "ptx.cuh"]),
+    (OUT, ["vidattn.cu"], ["vidattn.cu", "fwd_kernel.cuh", "classify.cuh", "ptx.cuh", "rope3d.cuh"]),
     # unit probes of the kernel's tensor-core steps, used only by the GPU tests
     (PROBES_OUT, ["probes.cu"], ["probes.cu", "fwd_kernel.cuh", "ptx.cuh"]),
 ]

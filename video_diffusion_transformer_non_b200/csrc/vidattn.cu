@@ -16,6 +16,7 @@
 #include "../../include/vidattn.h"
 #include "classify.cuh"
 #include "fwd_kernel.cuh"
+#include "rope3d.cuh"
 
 namespace vidattn {
 
@@ -75,6 +76,7 @@ struct DeviceInfo {
   bool ok = false;
   uint32_t attrs_set = 0;   // bit (kernel variant index) once its smem limit is raised
   int* err = nullptr;       // device address of g_device_error on this device
+  int rope_grid[4] = {};    // persistent grid of each rope3d variant (SMs x resident CTAs)
 };
 
 // Recently encoded tensor maps (per device): a call on the same buffers and
@@ -312,6 +314,53 @@ __global__ void selftest_timeout_kernel(int* err, unsigned long long timeout_ns)
   __syncwarp();
 }
 
+
+using RopeKernel = void (*)(const RopeParams);
+RopeKernel rope_variant(int i) {
+  switch (i) {
+    case 0: return rope3d_kernel<64, true>;
+    case 1: return rope3d_kernel<64, false>;
+    case 2: return rope3d_kernel<128, true>;
+    default: return rope3d_kernel<128, false>;
+  }
+}
+
+// SMs x resident CTAs of rope3d variant i on device dev (0 on failure).
+int rope_grid(int dev, int i) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& info = g_devices[dev];
+  if (info.rope_grid[i] == 0) {
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rope_variant(i), kRopeThreads, 0) !=
+            cudaSuccess)
+      return 0;
+    info.rope_grid[i] = sms * (per_sm > 0 ? per_sm : 1);
+  }
+  return info.rope_grid[i];
+}
+
+// Fills the per-column frequencies and the per-feature pairing tables.
+void rope_tables(RopeParams& p, int D, const int bands[3], double theta, bool half_split) {
+  int start = 0;
+  for (int a = 0; a < 3; ++a) {
+    const int d = bands[a], half = d / 2;
+    for (int k = 0; k < half; ++k) {
+      const int c = start / 2 + k;
+      p.freq[c] = std::pow(theta, -2.0 * k / d);
+      const int f0 = half_split ? start + k : start + 2 * k;
+      const int f1 = half_split ? start + k + half : start + 2 * k + 1;
+      p.col[f0] = p.col[f1] = static_cast<uint8_t>(c);
+      p.partner[f0] = static_cast<uint8_t>(f1);
+      p.partner[f1] = static_cast<uint8_t>(f0);
+      p.first[f0] = 1;
+      p.first[f1] = 0;
+    }
+    start += d;
+  }
+  (void)D;
+}
+
 }  // namespace
 }  // namespace vidattn
 
@@ -479,6 +528,65 @@ VIDATTN_API int vidattn_fwd_noalloc(const void* q, const void* k, const void* v,
                           stream);
   return launch_fwd<128>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
                          stream);
+}
+
+VIDATTN_API int vidattn_rope3d(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                               int B, int H, int S, int D,
+                               long long stride_b, long long stride_h, long long stride_s,
+                               int T, int Hg, int Wg, int token_offset,
+                               int d_t, int d_h, int d_w, double theta, int flags,
+                               vidattn_stream_t stream_) {
+  if (!q_in || !q_out || (k_in == nullptr) != (k_out == nullptr)) return VIDATTN_ERR_NULL;
+  if (D != 64 && D != 128) return VIDATTN_ERR_UNSUPPORTED_D;
+  if (flags & ~VIDATTN_ROPE_HALF_SPLIT) return VIDATTN_ERR_BAD_SHAPE;
+  const int n_tensors = k_in ? 2 : 1;
+  if (B < 1 || H < 1 || S < 1 || int64_t(n_tensors) * B * H >= (int64_t(1) << 31))
+    return VIDATTN_ERR_BAD_SHAPE;
+  if (T < 1 || Hg < 1 || Wg < 1 || token_offset < 0 ||
+      int64_t(token_offset) + int64_t(T) * Hg * Wg > S)
+    return VIDATTN_ERR_BAD_SHAPE;
+  const int bands[3] = {d_t, d_h, d_w};
+  for (int a = 0; a < 3; ++a)
+    if (bands[a] < 0 || bands[a] % 2) return VIDATTN_ERR_BAD_SHAPE;
+  if (d_t + d_h + d_w != D) return VIDATTN_ERR_BAD_SHAPE;
+  if (!std::isfinite(theta) || !(theta > 0.0)) return VIDATTN_ERR_BAD_SHAPE;
+  if (!aligned(q_in, 16) || !aligned(q_out, 16) || (k_in && (!aligned(k_in, 16) || !aligned(k_out, 16))))
+    return VIDATTN_ERR_MISALIGNED;
+  if (stride_b % 8 || stride_h % 8 || stride_s % 8) return VIDATTN_ERR_MISALIGNED;
+  int dev = 0;
+  int st = ensure_device(&dev);
+  if (st != VIDATTN_OK) return st;
+
+  const bool half_split = (flags & VIDATTN_ROPE_HALF_SPLIT) != 0;
+  RopeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.in[0] = static_cast<const uint16_t*>(q_in);
+  p.out[0] = static_cast<uint16_t*>(q_out);
+  p.in[1] = static_cast<const uint16_t*>(k_in ? k_in : q_in);
+  p.out[1] = static_cast<uint16_t*>(k_out ? k_out : q_out);
+  p.sb = stride_b;
+  p.sh = stride_h;
+  p.ss = stride_s;
+  p.n_slabs = n_tensors * B * H;
+  p.S = S;
+  p.div_bh = make_fastdiv(uint32_t(B) * uint32_t(H));
+  p.div_h = make_fastdiv(uint32_t(H));
+  p.n_video = T * Hg * Wg;
+  p.hw = Hg * Wg;
+  p.Hg = Hg;
+  p.Wg = Wg;
+  p.offset = token_offset;
+  p.col_h = d_t / 2;
+  p.col_w = (d_t + d_h) / 2;
+  rope_tables(p, D, bands, theta, half_split);
+
+  const int variant = (D == 128 ? 2 : 0) + (half_split ? 1 : 0);
+  const int grid_max = rope_grid(dev, variant);
+  if (grid_max <= 0) return VIDATTN_ERR_CUDA;
+  const int n_tiles = (S + kRopeTokens - 1) / kRopeTokens;
+  const int grid = n_tiles < grid_max ? n_tiles : grid_max;
+  rope_variant(variant)<<<grid, kRopeThreads, 0, reinterpret_cast<cudaStream_t>(stream_)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? VIDATTN_OK : VIDATTN_ERR_CUDA;
 }
 
 VIDATTN_API int vidattn_selftest_timeout(int timeout_us, vidattn_stream_t stream_) {

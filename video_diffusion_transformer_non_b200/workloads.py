@@ -21,6 +21,13 @@ Models on Accelerator Meshes, Fig. 1 and Tables 2 and 5: 480p and 720p
 Wan/HunyuanVideo grids, CogVideoX 720x480x49 with a 226-token T5 prompt), and
 stand in for them; the head counts and head dims are those of the named DiT
 families.
+
+The rotary-embedding conventions attached to each workload (the paper names
+3D RoPE per family but prints none) are taken from the families' public
+releases: Wan's split of a 128-wide head into t/h/w bands of 44/42/42
+features with theta 10000, CogVideoX's 16/24/24 of a 64-wide head with theta
+10000, HunyuanVideo's 16/56/56 with theta 256; all pair features 2k and 2k+1.
+Positions are the integer (t, h, w) indices of the latent grid.
 """
 from __future__ import annotations
 
@@ -41,6 +48,14 @@ class Workload:
     seed: int
     head_scaling: bool = False
     description: str = ""
+    # 3D rotary embedding of q and k ahead of the attention: the video tokens'
+    # (T, Hg, Wg) grid, where they start, the (d_t, d_h, d_w) feature bands,
+    # theta, and the pairing (True: features 2k, 2k+1; False: k, k + d/2)
+    rope_grid: tuple | None = None
+    rope_offset: int = 0
+    rope_bands: tuple | None = None
+    rope_theta: float = 10000.0
+    rope_interleaved: bool = True
 
     @property
     def S_q(self) -> int:
@@ -62,27 +77,33 @@ def _runs_total(runs):
 WORKLOADS = {
     "tiny": Workload(
         name="tiny", B=1, H=2, D=64, segments=None, S=512, seed=0,
-        description="B1 H2 D64 S512 (latent 2x16x16), one segment"),
+        description="B1 H2 D64 S512 (latent 2x16x16), one segment",
+        rope_grid=(2, 16, 16), rope_bands=(16, 24, 24)),
     "joint_small": Workload(
         name="joint_small", B=2, H=12, D=128,
         segments=((4096, 0), (256, 1), (37, 2)), S=4389, seed=1,
-        description="B2 H12 D128: 4096 video (4x32x32) + 256 text + 37 pad; ids video 0, text 1, pad 2"),
+        description="B2 H12 D128: 4096 video (4x32x32) + 256 text + 37 pad; ids video 0, text 1, pad 2",
+        rope_grid=(4, 32, 32), rope_bands=(44, 42, 42)),
     "video_480p": Workload(
         name="video_480p", B=1, H=40, D=128, segments=None, S=32760, seed=2,
         head_scaling=True,
-        description="B1 H40 D128 S32760 (21x30x52), one segment, q/k per-head scaled by U[0.5,2]"),
+        description="B1 H40 D128 S32760 (21x30x52), one segment, q/k per-head scaled by U[0.5,2]",
+        rope_grid=(21, 30, 52), rope_bands=(44, 42, 42)),
     "cogvideox_joint": Workload(
         name="cogvideox_joint", B=2, H=48, D=64,
         segments=((17550 + 226, 0), (16, 1)), S=17792, seed=3,
-        description="B2 H48 D64: 17550 video (13x30x45) + 226 text share id 0; 16 pad tokens id 1"),
+        description="B2 H48 D64: 17550 video (13x30x45) + 226 text share id 0; 16 pad tokens id 1",
+        rope_grid=(13, 30, 45), rope_bands=(16, 24, 24)),
     "video_720p": Workload(
         name="video_720p", B=1, H=24, D=128,
         segments=((118800, 0), (256, 1), (112, 2)), S=119168, seed=4,
-        description="B1 H24 D128: 118800 video (33x45x80) + 256 text + 112 pad; ids video 0, text 1, pad 2"),
+        description="B1 H24 D128: 118800 video (33x45x80) + 256 text + 112 pad; ids video 0, text 1, pad 2",
+        rope_grid=(33, 45, 80), rope_bands=(16, 56, 56), rope_theta=256.0),
 }
 
 for _w in WORKLOADS.values():
     assert _w.segments is None or _runs_total(_w.segments) == _w.S, _w.name
+    assert _w.rope_offset + int(np.prod(_w.rope_grid)) <= _w.S and sum(_w.rope_bands) == _w.D, _w.name
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
