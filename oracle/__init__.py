@@ -9,7 +9,10 @@ this module compiles it with gcc and marshals numpy arrays through ctypes.
 What it computes, with citations, is written at the top of ``attn_oracle.c``:
 exact softmax(scale * Q K^T masked by segment-id equality) V, plus the natural
 log-sum-exp of each row, with empty rows giving out = 0 and lse = -inf; with
-causal=True a key is also limited to j <= i + (S_kv - S_q).
+causal=True a key is also limited to j <= i + (S_kv - S_q); with a ``window``
+(a 3D neighbourhood: per-token packed coordinates t << 22 | h << 11 | w, an odd
+window size and the volume extent per axis, centred or clamped) a key must
+also lie in the query's window.
 
 Inputs are bf16 bit patterns as ``numpy.uint16`` arrays in [B,H,S,D] order and
 int32 segment ids in [B,S] order (or None for a single segment).
@@ -40,23 +43,37 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def _declare(lib):
+    """Argument and result types of the library's entry points."""
+    p = ctypes.c_void_p
+    L = ctypes.c_long
+    lib.oracle_attn_fwd_f64.argtypes = [p, p, p, p, p, p, p, L, L, L, L, L,
+                                        ctypes.c_double, ctypes.c_int, ctypes.c_int]
+    lib.oracle_attn_fwd_f64.restype = ctypes.c_int
+    lib.oracle_attn_rows_f64.argtypes = [p, p, p, p, p, p, L, p, p, L, L, L, L, L,
+                                         ctypes.c_double, ctypes.c_int, ctypes.c_int]
+    lib.oracle_attn_rows_f64.restype = ctypes.c_int
+    lib.oracle_attn_probs_f64.argtypes = [p, p, p, p, p, L, L, L, L, L, ctypes.c_double,
+                                          ctypes.c_int]
+    lib.oracle_attn_probs_f64.restype = ctypes.c_int
+    W = [p, p, p, p, ctypes.c_int]     # coord_q, coord_kv, size[3], extent[3], clamped
+    lib.oracle_attn_win_fwd_f64.argtypes = [p, p, p, p, p] + W + [
+        p, p, L, L, L, L, L, ctypes.c_double, ctypes.c_int, ctypes.c_int]
+    lib.oracle_attn_win_fwd_f64.restype = ctypes.c_int
+    lib.oracle_attn_win_rows_f64.argtypes = [p, p, p, p, p] + W + [
+        p, L, p, p, L, L, L, L, L, ctypes.c_double, ctypes.c_int, ctypes.c_int]
+    lib.oracle_attn_win_rows_f64.restype = ctypes.c_int
+    lib.oracle_attn_win_probs_f64.argtypes = [p, p, p, p] + W + [
+        p, L, L, L, L, L, ctypes.c_double, ctypes.c_int]
+    lib.oracle_attn_win_probs_f64.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
         build()
-        lib = ctypes.CDLL(_LIB_PATH)
-        p = ctypes.c_void_p
-        L = ctypes.c_long
-        lib.oracle_attn_fwd_f64.argtypes = [p, p, p, p, p, p, p, L, L, L, L, L,
-                                            ctypes.c_double, ctypes.c_int, ctypes.c_int]
-        lib.oracle_attn_fwd_f64.restype = ctypes.c_int
-        lib.oracle_attn_rows_f64.argtypes = [p, p, p, p, p, p, L, p, p, L, L, L, L, L,
-                                             ctypes.c_double, ctypes.c_int, ctypes.c_int]
-        lib.oracle_attn_rows_f64.restype = ctypes.c_int
-        lib.oracle_attn_probs_f64.argtypes = [p, p, p, p, p, L, L, L, L, L, ctypes.c_double,
-                                              ctypes.c_int]
-        lib.oracle_attn_probs_f64.restype = ctypes.c_int
-        _lib = lib
+        _lib = _declare(ctypes.CDLL(_LIB_PATH))
     return _lib
 
 
@@ -81,13 +98,39 @@ def _check_inputs(q, k, v, seg_q, seg_kv):
     return B, H, S_q, S_kv, D
 
 
-def attn_fwd(q, k, v, seg_q=None, seg_kv=None, scale=None, nthreads=0, causal=False):
+def _window_args(window, B, S_q, S_kv):
+    """window: dict(coord_q int32 [B,S_q], coord_kv int32 [B,S_kv], size (kt,kh,kw),
+    extent (T,Hg,Wg), clamped bool).  Returns the ctypes arguments and the
+    arrays they point to (kept alive by the caller)."""
+    cq = np.ascontiguousarray(window["coord_q"], dtype=np.int32)
+    ck = np.ascontiguousarray(window["coord_kv"], dtype=np.int32)
+    if cq.shape != (B, S_q) or ck.shape != (B, S_kv):
+        raise ValueError("window coordinates must be int32 [B,S_q] and [B,S_kv]")
+    size = np.ascontiguousarray(window["size"], dtype=np.int64)
+    extent = np.ascontiguousarray(window["extent"], dtype=np.int64)
+    if size.shape != (3,) or extent.shape != (3,):
+        raise ValueError("window size and extent have one entry per axis (t, h, w)")
+    keep = (cq, ck, size, extent)
+    return [_ptr(cq), _ptr(ck), _ptr(size), _ptr(extent), int(bool(window["clamped"]))], keep
+
+
+def attn_fwd(q, k, v, seg_q=None, seg_kv=None, scale=None, nthreads=0, causal=False,
+             window=None):
     """All rows.  Returns (out float64 [B,H,S_q,D], lse float64 [B,H,S_q])."""
     B, H, S_q, S_kv, D = _check_inputs(q, k, v, seg_q, seg_kv)
     if scale is None:
         scale = 1.0 / np.sqrt(D)
     out = np.empty((B, H, S_q, D), np.float64)
     lse = np.empty((B, H, S_q), np.float64)
+    if window is not None:
+        wargs, _keep = _window_args(window, B, S_q, S_kv)
+        rc = _load().oracle_attn_win_fwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(seg_q),
+                                             _ptr(seg_kv), *wargs, _ptr(out), _ptr(lse),
+                                             B, H, S_q, S_kv, D, float(scale),
+                                             int(bool(causal)), int(nthreads))
+        if rc != 0:
+            raise RuntimeError(f"oracle_attn_win_fwd_f64 failed with code {rc}")
+        return out, lse
     rc = _load().oracle_attn_fwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv),
                                      _ptr(out), _ptr(lse), B, H, S_q, S_kv, D,
                                      float(scale), int(bool(causal)), int(nthreads))
@@ -96,7 +139,8 @@ def attn_fwd(q, k, v, seg_q=None, seg_kv=None, scale=None, nthreads=0, causal=Fa
     return out, lse
 
 
-def attn_rows(q, k, v, rows, seg_q=None, seg_kv=None, scale=None, nthreads=0, causal=False):
+def attn_rows(q, k, v, rows, seg_q=None, seg_kv=None, scale=None, nthreads=0, causal=False,
+              window=None):
     """Selected rows.  rows: int64 [n,3] of (b, h, i).
     Returns (out float64 [n,D], lse float64 [n])."""
     B, H, S_q, S_kv, D = _check_inputs(q, k, v, seg_q, seg_kv)
@@ -106,6 +150,15 @@ def attn_rows(q, k, v, rows, seg_q=None, seg_kv=None, scale=None, nthreads=0, ca
     n = rows.shape[0]
     out = np.empty((n, D), np.float64)
     lse = np.empty((n,), np.float64)
+    if window is not None:
+        wargs, _keep = _window_args(window, B, S_q, S_kv)
+        rc = _load().oracle_attn_win_rows_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(seg_q),
+                                              _ptr(seg_kv), *wargs, _ptr(rows), n, _ptr(out),
+                                              _ptr(lse), B, H, S_q, S_kv, D, float(scale),
+                                              int(bool(causal)), int(nthreads))
+        if rc != 0:
+            raise RuntimeError(f"oracle_attn_win_rows_f64 failed with code {rc}")
+        return out, lse
     rc = _load().oracle_attn_rows_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(seg_q), _ptr(seg_kv),
                                       _ptr(rows), n, _ptr(out), _ptr(lse),
                                       B, H, S_q, S_kv, D, float(scale), int(bool(causal)),
@@ -115,7 +168,7 @@ def attn_rows(q, k, v, rows, seg_q=None, seg_kv=None, scale=None, nthreads=0, ca
     return out, lse
 
 
-def attn_probs(q, k, seg_q=None, seg_kv=None, scale=None, causal=False):
+def attn_probs(q, k, seg_q=None, seg_kv=None, scale=None, causal=False, window=None):
     """Softmax weights [B,H,S_q,S_kv] (small inputs only); masked entries are 0."""
     B, H, S_q, D = q.shape
     S_kv = k.shape[2]
@@ -123,6 +176,14 @@ def attn_probs(q, k, seg_q=None, seg_kv=None, scale=None, causal=False):
     if scale is None:
         scale = 1.0 / np.sqrt(D)
     probs = np.empty((B, H, S_q, S_kv), np.float64)
+    if window is not None:
+        wargs, _keep = _window_args(window, B, S_q, S_kv)
+        rc = _load().oracle_attn_win_probs_f64(_ptr(q), _ptr(k), _ptr(seg_q), _ptr(seg_kv),
+                                               *wargs, _ptr(probs), B, H, S_q, S_kv, D,
+                                               float(scale), int(bool(causal)))
+        if rc != 0:
+            raise RuntimeError(f"oracle_attn_win_probs_f64 failed with code {rc}")
+        return probs
     rc = _load().oracle_attn_probs_f64(_ptr(q), _ptr(k), _ptr(seg_q), _ptr(seg_kv),
                                        _ptr(probs), B, H, S_q, S_kv, D, float(scale),
                                        int(bool(causal)))
