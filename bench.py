@@ -155,7 +155,11 @@ def oracle_rows_throughput(w, inputs, n_rows, seed=0, causal=False):
     rows = np.stack([rng.integers(0, w.B, n_rows), rng.integers(0, w.H, n_rows),
                      rng.integers(0, w.S_q, n_rows)], 1).astype(np.int64)
     lim = (lambda i: i + 1 + w.S_kv - w.S_q) if causal else (lambda i: w.S_kv)
-    if inputs["seg_q"] is not None:
+    from video_diffusion_transformer_non_b200 import workloads as wl
+    window = wl.window_of(w) if w.window is not None else None
+    if window is not None:
+        allowed = wl.window_row_counts(w, rows[:, 2])
+    elif inputs["seg_q"] is not None:
         sq, sk = inputs["seg_q"], inputs["seg_kv"]
         allowed = np.array([int(np.count_nonzero(sk[b, :max(0, lim(i))] == sq[b, i]))
                             for b, _, i in rows])
@@ -164,7 +168,7 @@ def oracle_rows_throughput(w, inputs, n_rows, seed=0, causal=False):
     threads = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
     oracle.attn_rows(inputs["q"], inputs["k"], inputs["v"], rows, inputs["seg_q"],
-                     inputs["seg_kv"], w.scale, nthreads=threads, causal=causal)
+                     inputs["seg_kv"], w.scale, nthreads=threads, causal=causal, window=window)
     dt = time.perf_counter() - t0
     flops = 4.0 * w.D * float(allowed.sum())
     return flops / dt / 1e12, dt, threads
@@ -237,7 +241,11 @@ def rope_algorithmic_bytes(w) -> int:
 
 
 def workload_config(w, causal=False, rope=False):
-    return {"workload": w.name + ("_causal" if causal else "") + ("_rope" if rope else ""),
+    extra = {}
+    if w.window is not None:
+        extra = {"window": list(w.window), "volume": list(w.rope_grid),
+                 "window_clamped": w.window_clamped, "token_order": "raster"}
+    return {**extra, "workload": w.name + ("_causal" if causal else "") + ("_rope" if rope else ""),
             "B": w.B, "H": w.H, "S_q": w.S_q, "S_kv": w.S_kv, "D": w.D, "causal": causal,
             "segments": None if w.segments is None else [list(r) for r in w.segments],
             "description": w.description,
@@ -310,6 +318,14 @@ def main(argv=None):
     lse = torch.empty((w.B, w.H, w.S_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
+    windowed = w.window is not None
+    if windowed and (args.causal or args.rope):
+        ap.error("window workloads run without --causal and --rope")
+    if windowed:
+        win = wl.window_of(w)
+        cq = torch.from_numpy(win["coord_q"].copy()).to(dev)
+        ck = torch.from_numpy(win["coord_kv"].copy()).to(dev)
+        win_flags = binding.VIDATTN_WINDOW_CLAMPED if w.window_clamped else 0
 
     flags = binding.VIDATTN_CAUSAL if args.causal else 0
     use_rope = args.rope
@@ -337,6 +353,14 @@ def main(argv=None):
             if timed:
                 e[1].record(stream)
                 rope_ev.append(e)
+        if windowed:
+            st = lib.vidattn_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), cq.data_ptr(),
+                                        ck.data_ptr(), out.data_ptr(), lse.data_ptr(), w.B, w.H,
+                                        w.S_q, w.S_kv, w.D, w.scale, *w.window, *w.rope_grid,
+                                        win_flags, sh)
+            if st != 0:
+                raise RuntimeError(binding.status_string(st))
+            return
         st = lib.vidattn_fwd_ex(qa.data_ptr(), ka.data_ptr(), v.data_ptr(),
                                 None if sq is None else sq.data_ptr(),
                                 None if sk is None else sk.data_ptr(),
@@ -392,20 +416,27 @@ def main(argv=None):
         hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
         ptr = lambda t: None if t is None else t.data_ptr()
 
-        def e2e_step_rope():
+        hcq = pin(win["coord_q"]) if windowed else None
+        hck = pin(win["coord_kv"]) if windowed else None
+
+        def e2e_step_api():
+            # pinned inputs in, the step's C-ABI calls, outputs back
             q.copy_(hq.view(torch.bfloat16), non_blocking=True)
             k.copy_(hk.view(torch.bfloat16), non_blocking=True)
             v.copy_(hv.view(torch.bfloat16), non_blocking=True)
             if hsq is not None:
                 sq.copy_(hsq, non_blocking=True)
                 sk.copy_(hsk, non_blocking=True)
+            if windowed:
+                cq.copy_(hcq, non_blocking=True)
+                ck.copy_(hck, non_blocking=True)
             step()
             hout.copy_(out.view(torch.int16), non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
 
         def e2e_step():
-            if use_rope:
-                return e2e_step_rope()
+            if use_rope or windowed:
+                return e2e_step_api()
             st = lib.vidattn_fwd_host(ptr(hq), ptr(hk), ptr(hv), ptr(hsq), ptr(hsk), ptr(hout),
                                       ptr(hlse), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                       ptr(sq), ptr(sk), out.data_ptr(), lse.data_ptr(),
@@ -427,7 +458,8 @@ def main(argv=None):
         torch.cuda.synchronize(dev)
         barrier()
         e_ms = rank_max(e0.elapsed_time(e1))
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsq, hsk) if t is not None)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsq, hsk, hcq, hck)
+                  if t is not None)
         d2h = hout.numel() * 2 + hlse.numel() * 4
         e2e = {"value": weak_scaling_value(flops_step, n_e2e, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -478,7 +510,7 @@ def main(argv=None):
             "hbm_gbs": algorithmic_bytes(w) / (kernel_ms * 1e-3) / 1e9,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (binding.kernels_per_call(
-                sq, sk, w.B, w.H, w.S_q, w.S_kv, w.D) + (1 if use_rope else 0)),
+                sq, sk, w.B, w.H, w.S_q, w.S_kv, w.D) + (1 if use_rope or windowed else 0)),
             "rope3d": rope,
             "clocks": clocks,
         }

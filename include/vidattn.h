@@ -119,6 +119,54 @@ VIDATTN_API int vidattn_fwd_ex(const void* q, const void* k, const void* v,
                                int B, int H, int S_q, int S_kv, int D, float scale, int flags,
                                vidattn_stream_t stream);
 
+/* Flags of vidattn_fwd_window. */
+#define VIDATTN_WINDOW_CLAMPED 1   /* windows shifted inside the volume at its borders */
+
+/* Packs a token's coordinates for vidattn_fwd_window (t < 1024, h, w < 2048). */
+#define VIDATTN_COORD(t, h, w) \
+  ((int32_t)(((uint32_t)(t) << 22) | ((uint32_t)(h) << 11) | (uint32_t)(w)))
+
+/*
+ * vidattn_fwd_window — 3D neighbourhood (windowed) attention: the attention of
+ * vidattn_fwd with each query limited to the keys in a window around its own
+ * position in the video volume.  The vidax paper (Appendix A, Table 4, group 4
+ * "Memory, Tiling & Execution Graphs", rows on the LTX-2.5 VAE decoder) runs
+ * 3D neighbourhood attention with an 11 x 11 x 11 window and gives no
+ * formula; this is the window of neighbourhood attention (Hassani et al.,
+ * "Neighborhood Attention Transformer", CVPR 2023):
+ *
+ *   every token carries coordinates (t, h, w) in a T x Hg x Wg volume, given
+ *   per token as VIDATTN_COORD(t, h, w) in coord_q [B,S_q] and coord_kv
+ *   [B,S_kv] (int32, device, 4-byte aligned; any token order).  On each axis
+ *   a window of odd size k (win_t, win_h, win_w) starts at c - (k-1)/2 for a
+ *   query at coordinate c, or, with VIDATTN_WINDOW_CLAMPED, at that start
+ *   pushed into [0, extent - k] so that queries at the borders still see k
+ *   keys on that axis.  Query i sees key j iff on every axis
+ *   start <= c_j <= start + k - 1; out and lse are vidattn_fwd's over those
+ *   keys (a row that sees none: out 0, lse -inf).
+ *
+ *   win_t, win_h, win_w   odd, >= 1
+ *   T, Hg, Wg             volume extents, 1..1024, 1..2048, 1..2048; every
+ *                         coordinate must be below its extent
+ *   S_kv                  <= 262144 (the key tiles of a CTA are listed in
+ *                         shared memory)
+ *   flags                 0 or VIDATTN_WINDOW_CLAMPED
+ *   the rest              as vidattn_fwd.
+ *
+ * Key tiles (128 keys) whose coordinate box misses every window of a CTA's
+ * 256 queries are never loaded; tiles inside every window skip the mask.  Two
+ * kernels per call (tile boxes, then the attention); the tile boxes use the
+ * scratch of vidattn_fwd (per device and stream).  Errors: NULL coordinates
+ * return VIDATTN_ERR_NULL; bad window sizes, extents, S_kv or flag bits
+ * VIDATTN_ERR_BAD_SHAPE; otherwise as vidattn_fwd.
+ */
+VIDATTN_API int vidattn_fwd_window(const void* q, const void* k, const void* v,
+                                   const int32_t* coord_q, const int32_t* coord_kv,
+                                   void* out, float* lse,
+                                   int B, int H, int S_q, int S_kv, int D, float scale,
+                                   int win_t, int win_h, int win_w, int T, int Hg, int Wg,
+                                   int flags, vidattn_stream_t stream);
+
 /*
  * vidattn_fwd_host — the same operation on HOST buffers, for callers whose
  * data lives in host memory.  h_* are host pointers (pinned memory gives

@@ -32,6 +32,7 @@ def header_names():
 def test_header_declares_the_entry_points():
     names = set(header_names())
     assert {"vidattn_fwd", "vidattn_fwd_ex", "vidattn_fwd_host", "vidattn_status_string", "vidattn_device_status",
+            "vidattn_rope3d", "vidattn_fwd_window",
             "vidattn_kernels_per_call", "vidattn_release", "vidattn_version",
             "vidattn_selftest_timeout"} <= names
     assert set(binding.exported_symbols()) == names
@@ -164,3 +165,27 @@ def test_rope3d_q_only_is_accepted_by_the_checks(lib):
     """k_in and k_out both NULL passes the argument checks (then needs a GPU)."""
     st = rope(lib, k=None, ko=None)
     assert st in (OK, CUDA, NO_DEVICE)
+
+
+def win(lib, q=A, k=A, v=A, cq=A + 0x1000, ck=A + 0x2000, out=A, lse=A, B=1, H=2, Sq=512, Skv=512,
+        D=128, scale=0.125, size=(3, 5, 5), ext=(2, 16, 16), flags=0):
+    return lib.vidattn_fwd_window(q, k, v, cq, ck, out, lse, B, H, Sq, Skv, D, scale, *size, *ext,
+                                  flags, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(cq=None), NULL), (dict(ck=None), NULL), (dict(q=None), NULL),
+    (dict(D=96), BAD_D), (dict(flags=2), BAD_SHAPE), (dict(flags=-1), BAD_SHAPE),
+    (dict(size=(2, 5, 5)), BAD_SHAPE), (dict(size=(3, 0, 5)), BAD_SHAPE),
+    (dict(size=(3, 5, -1)), BAD_SHAPE), (dict(ext=(0, 16, 16)), BAD_SHAPE),
+    (dict(ext=(1025, 16, 16)), BAD_SHAPE), (dict(ext=(2, 2049, 16)), BAD_SHAPE),
+    (dict(ext=(2, 16, 2049)), BAD_SHAPE), (dict(Skv=262145), BAD_SHAPE),
+    (dict(scale=float("nan")), BAD_SHAPE), (dict(B=0), BAD_SHAPE),
+    (dict(cq=A + 2), MISALIGNED), (dict(q=A + 8), MISALIGNED),
+])
+def test_window_argument_errors_return_before_any_launch(lib, kw, expect):
+    assert win(lib, **kw) == expect
+
+
+def test_window_empty_query_is_a_no_op(lib):
+    assert win(lib, Sq=0) == OK

@@ -56,6 +56,9 @@ def load_library():
     lib.vidattn_kernels_per_call.restype = i32
     lib.vidattn_selftest_timeout.argtypes = [i32, p]
     lib.vidattn_selftest_timeout.restype = i32
+    lib.vidattn_fwd_window.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, f32,
+                                       i32, i32, i32, i32, i32, i32, i32, p]
+    lib.vidattn_fwd_window.restype = i32
     i64, f64 = ctypes.c_longlong, ctypes.c_double
     lib.vidattn_rope3d.argtypes = [p, p, p, p, i32, i32, i32, i32, i64, i64, i64,
                                    i32, i32, i32, i32, i32, i32, i32, f64, i32, p]
@@ -210,3 +213,33 @@ def rope3d(q, k=None, grid=None, bands=None, theta=10000.0, interleaved=True, to
     if st != VIDATTN_OK:
         raise RuntimeError(f"vidattn_rope3d failed: {status_string(st)} ({st})")
     return out_q, out_k
+
+
+VIDATTN_WINDOW_CLAMPED = 1
+
+
+def vidattn_fwd_window(q, k, v, coord_q, coord_kv, out, lse, B, H, S_q, S_kv, D, scale,
+                       win_t, win_h, win_w, T, Hg, Wg, flags, stream=None) -> int:
+    """Enqueue 3D neighbourhood attention on ``stream``.  Returns the status."""
+    return load_library().vidattn_fwd_window(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(coord_q), _ptr(coord_kv), _ptr(out), _ptr(lse),
+        int(B), int(H), int(S_q), int(S_kv), int(D), float(scale), int(win_t), int(win_h),
+        int(win_w), int(T), int(Hg), int(Wg), int(flags), _stream(stream))
+
+
+def attention_window(q, k, v, coord_q, coord_kv, size, extent, clamped=True, scale=None,
+                     stream=None):
+    """3D neighbourhood attention.  coord_*: int32 [B,S] packed t << 22 | h << 11 | w;
+    size = (win_t, win_h, win_w), odd; extent = (T, Hg, Wg).  Returns (out, lse)."""
+    import torch
+    B, H, S_q, D = q.shape
+    S_kv = k.shape[2]
+    if scale is None:
+        scale = D ** -0.5
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S_q), dtype=torch.float32, device=q.device)
+    st = vidattn_fwd_window(q, k, v, coord_q, coord_kv, out, lse, B, H, S_q, S_kv, D, scale,
+                            *size, *extent, VIDATTN_WINDOW_CLAMPED if clamped else 0, stream)
+    if st != VIDATTN_OK:
+        raise RuntimeError(f"vidattn_fwd_window failed: {status_string(st)} ({st})")
+    return out, lse

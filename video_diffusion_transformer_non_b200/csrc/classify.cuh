@@ -48,4 +48,60 @@ __global__ void __launch_bounds__(128) seg_tile_classify_kernel(
   }
 }
 
+// 3D neighbourhood windows (vidattn_fwd_window): for every (b, 128-token
+// tile) of coord_q and coord_kv, the bounding box of the tile's (t, h, w)
+// coordinates, int4 {t_lo | t_hi << 16, h_lo | h_hi << 16, w_lo | w_hi << 16, 0}
+// (coordinates packed per token as t << 22 | h << 11 | w).  The attention
+// kernel skips a key tile whose box misses the union of its queries' windows
+// and takes the unmasked path where the box lies inside every query's window.
+// Launch shape as seg_tile_classify_kernel.
+__global__ void __launch_bounds__(128) win_tile_bbox_kernel(
+    const int32_t* __restrict__ coord_q, const int32_t* __restrict__ coord_kv,
+    int4* __restrict__ q_box, int4* __restrict__ kv_box, int S_q, int S_kv) {
+  const int which = blockIdx.z;
+  const int b = blockIdx.y;
+  const int tile = blockIdx.x;
+  const int S = which ? S_kv : S_q;
+  const int n_tiles = (S + kSegTile - 1) / kSegTile;
+  if (tile >= n_tiles) return;
+  const int32_t* coord = (which ? coord_kv : coord_q) + static_cast<int64_t>(b) * S;
+  const int idx = tile * kSegTile + threadIdx.x;
+  int lo[3] = {INT_MAX, INT_MAX, INT_MAX}, hi[3] = {INT_MIN, INT_MIN, INT_MIN};
+  if (idx < S) {
+    const uint32_t c = static_cast<uint32_t>(__ldg(coord + idx));
+    lo[0] = hi[0] = int(c >> 22);
+    lo[1] = hi[1] = int((c >> 11) & 2047u);
+    lo[2] = hi[2] = int(c & 2047u);
+  }
+#pragma unroll
+  for (int a = 0; a < 3; ++a) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo[a] = min(lo[a], __shfl_xor_sync(0xffffffffu, lo[a], o));
+      hi[a] = max(hi[a], __shfl_xor_sync(0xffffffffu, hi[a], o));
+    }
+  }
+  __shared__ int s_lo[3][4], s_hi[3][4];
+  const int warp = threadIdx.x / 32;
+  if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      s_lo[a][warp] = lo[a];
+      s_hi[a][warp] = hi[a];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int packed[3];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      const int l = min(min(s_lo[a][0], s_lo[a][1]), min(s_lo[a][2], s_lo[a][3]));
+      const int h = max(max(s_hi[a][0], s_hi[a][1]), max(s_hi[a][2], s_hi[a][3]));
+      packed[a] = l | (h << 16);
+    }
+    int4* dst = (which ? kv_box : q_box) + static_cast<int64_t>(b) * n_tiles + tile;
+    *dst = make_int4(packed[0], packed[1], packed[2], 0);
+  }
+}
+
 }  // namespace vidattn

@@ -54,8 +54,15 @@ constexpr int kMaxListedTiles = 2048;
 struct FwdParams {
   const int32_t* seg_q;     // [B,S_q] or null
   const int32_t* seg_kv;    // [B,S_kv] or null
-  const int4* q_sum;        // [B,n_q_tiles] {min,max,uniform,0}; null without ids
+  // ids: [B,n_q_tiles] {min,max,uniform,0}; window: the tiles' coordinate
+  // boxes (win_tile_bbox_kernel); null with neither
+  const int4* q_sum;
   const int4* kv_sum;       // [B,n_kv_tiles]
+  // 3D neighbourhood window (vidattn_fwd_window), or coord_q == null: per-token
+  // coordinates t << 22 | h << 11 | w, window size and volume extent per axis
+  const int32_t* coord_q;   // [B,S_q]
+  const int32_t* coord_kv;  // [B,S_kv]
+  int win_size[3], win_extent[3], win_clamped;
   uint16_t* out;            // bf16 [B,H,S_q,D]
   float* lse;               // fp32 [B,H,S_q]
   int* err;                 // device error word (bit kErrTimeout: a wait timed out)
@@ -96,7 +103,11 @@ struct FwdCfg {
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;   // tmem addr, abort flag
   static constexpr int kOffWarpCnt = kOffMisc + 16;         // 12 ints (list building)
   static constexpr int kOffList = kOffWarpCnt + 64;         // active key tiles
-  static constexpr int kSmemBytes = kOffList + 4 * kMaxListedTiles + 1024;  // + alignment slack
+  // per softmax warp: the ids or window coordinates of the 128 keys of the
+  // masked key tile it is working on (read as int4: 16-byte aligned)
+  static constexpr int kOffKinfo = (kOffList + 4 * kMaxListedTiles + 127) & ~127;
+  static_assert(kOffKinfo % 16 == 0, "int4 reads of the key-info slots");
+  static constexpr int kSmemBytes = kOffKinfo + 8 * kBN * 4 + 1024;  // + alignment slack
   // P in its own tensor-memory columns (D = 64, where they fit) instead of
   // over the first half of S: the next Q K^T of a tile need not wait for
   // the P V that reads its P.
@@ -166,6 +177,177 @@ struct KvWalk {
   }
 };
 
+// ------------------------------------------------- 3D neighbourhood window
+// On each axis the window of a query at coordinate c spans
+// [start, start + size - 1], start = c - (size - 1) / 2, pushed into
+// [0, extent - size] when clamped (every query then sees size keys per axis).
+__device__ __forceinline__ int win_start(int c, int size, int extent, int clamped) {
+  int s = c - (size - 1) / 2;
+  if (clamped) s = max(min(s, extent - size), 0);
+  return s;
+}
+__device__ __forceinline__ int coord_axis(uint32_t c, int a) {
+  return a == 0 ? int(c >> 22) : (a == 1 ? int((c >> 11) & 2047u) : int(c & 2047u));
+}
+// Window starts of one query row.
+struct WinRow {
+  int s[3];
+};
+__device__ __forceinline__ WinRow win_row(const FwdParams& p, uint32_t qc) {
+  WinRow r;
+#pragma unroll
+  for (int a = 0; a < 3; ++a)
+    r.s[a] = win_start(coord_axis(qc, a), p.win_size[a], p.win_extent[a], p.win_clamped);
+  return r;
+}
+__device__ __forceinline__ bool win_has(const FwdParams& p, const WinRow& r, uint32_t kc) {
+  bool in = true;
+#pragma unroll
+  for (int a = 0; a < 3; ++a)
+    in = in && uint32_t(coord_axis(kc, a) - r.s[a]) < uint32_t(p.win_size[a]);
+  return in;
+}
+// Tile boxes: field a of the int4 packs lo | hi << 16 for axis a.
+__device__ __forceinline__ int box_lo(int4 b, int a) {
+  return (a == 0 ? b.x : (a == 1 ? b.y : b.z)) & 0xFFFF;
+}
+__device__ __forceinline__ int box_hi(int4 b, int a) {
+  return (a == 0 ? b.x : (a == 1 ? b.y : b.z)) >> 16;
+}
+// Could some query of the two Q tiles (boxes qa, qb) see some key of a K tile
+// with box kb?  (Its box meets the union of their windows on every axis.)
+__device__ __forceinline__ bool win_tile_meets(const FwdParams& p, int4 qa, int4 qb, int4 kb) {
+  bool meets = true;
+#pragma unroll
+  for (int a = 0; a < 3; ++a) {
+    const int qlo = min(box_lo(qa, a), box_lo(qb, a)), qhi = max(box_hi(qa, a), box_hi(qb, a));
+    const int u_lo = win_start(qlo, p.win_size[a], p.win_extent[a], p.win_clamped);
+    const int u_hi = win_start(qhi, p.win_size[a], p.win_extent[a], p.win_clamped) +
+                     p.win_size[a] - 1;
+    meets = meets && box_hi(kb, a) >= u_lo && box_lo(kb, a) <= u_hi;
+  }
+  return meets;
+}
+// Does every query of a Q tile (box qa) see every key of a K tile (box kb)?
+// (The K box lies inside the intersection of the queries' windows.)
+__device__ __forceinline__ bool win_tile_full(const FwdParams& p, int4 qa, int4 kb) {
+  bool full = true;
+#pragma unroll
+  for (int a = 0; a < 3; ++a) {
+    const int i_lo = win_start(box_hi(qa, a), p.win_size[a], p.win_extent[a], p.win_clamped);
+    const int i_hi = win_start(box_lo(qa, a), p.win_size[a], p.win_extent[a], p.win_clamped) +
+                     p.win_size[a] - 1;
+    full = full && box_lo(kb, a) >= i_lo && box_hi(kb, a) <= i_hi;
+  }
+  return full;
+}
+
+// Sets bits [lo, hi) of a 128-bit mask.
+__device__ __forceinline__ void set_bit_range(uint32_t (&mb)[4], int lo, int hi) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int a = max(lo - 32 * k, 0), e = min(hi - 32 * k, 32);
+    if (a < e) mb[k] |= (e == 32 ? 0xFFFFFFFFu : ((1u << e) - 1u)) & ~((1u << a) - 1u);
+  }
+}
+
+constexpr int kMaxRuns = 16;   // runs per key tile handled run by run
+
+// The mask of one query row over a masked key tile, bit x of word x/32 set
+// when key x of the tile is visible: x < n_lim (the key exists and lies
+// within the causal limit) and the key has the row's id (mode 1) or lies in
+// its window (mode 2: window starts ws0..2, sizes k0..2).  kinfo: the 128
+// keys' ids or coordinates, staged in this warp's shared memory by the
+// caller (unused in mode 0).  Called by the whole warp.
+//
+// The keys of a tile fall into runs: consecutive keys with one id, or with
+// one (t, h) and consecutive w (a row of the volume in raster order).  A
+// row's visible keys in a run are one contiguous range, so with few runs the
+// mask is built run by run; otherwise key by key.
+__device__ __forceinline__ uint4 tile_mask(const int32_t* kinfo, int mode, int my_seg, int ws0,
+                                        int ws1, int ws2, int k0, int k1, int k2, int n_lim) {
+  const int lane = threadIdx.x & 31;
+  uint32_t mb[4] = {0u, 0u, 0u, 0u};
+  if (mode == 0) {
+    set_bit_range(mb, 0, n_lim);
+    return make_uint4(mb[0], mb[1], mb[2], mb[3]);
+  }
+  const bool ids = mode == 1;
+  // run starts (the same for every row of the warp)
+  uint32_t starts[4];
+  int n_runs = 0;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int x = lane + 32 * m;
+    const int32_t cur = kinfo[x];
+    const int32_t prev = kinfo[x > 0 ? x - 1 : 0];
+    const bool cont = ids ? (prev == cur)
+                          : (uint32_t(cur) == uint32_t(prev) + 1u && (cur & 2047) != 0);
+    starts[m] = __ballot_sync(0xFFFFFFFFu, x == 0 || !cont);
+    n_runs += __popc(starts[m]);
+  }
+  if (n_runs <= kMaxRuns) {
+    // walk the runs in order: [xa, xb)
+    uint32_t rest[4] = {starts[0] & ~1u, starts[1], starts[2], starts[3]};
+    int xa = 0;
+    for (int r = 0; r < n_runs; ++r) {
+      int xb = kBN;
+#pragma unroll
+      for (int k = 3; k >= 0; --k)
+        if (rest[k]) xb = 32 * k + __ffs(rest[k]) - 1;
+      const int32_t c0 = kinfo[xa];
+      if (ids) {
+        if (c0 == my_seg) set_bit_range(mb, xa, xb);
+      } else {
+        const uint32_t u = uint32_t(c0);
+        if (uint32_t(int(u >> 22) - ws0) < uint32_t(k0) &&
+            uint32_t(int((u >> 11) & 2047u) - ws1) < uint32_t(k1)) {
+          const int w0 = int(u & 2047u);
+          const int lo = xa + max(ws2 - w0, 0);
+          const int hi = xa + min(ws2 + k2 - w0, xb - xa);
+          if (lo < hi) set_bit_range(mb, lo, hi);
+        }
+      }
+      // clear the next run's start bit (selects: no dynamic register index)
+      const uint32_t clear = ~(1u << (xb & 31));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rest[k] &= ((xb >> 5) == k) ? clear : 0xFFFFFFFFu;
+      xa = xb;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t bits = 0u;
+#pragma unroll
+      for (int x = 0; x < 32; x += 4) {
+        const int4 v = *reinterpret_cast<const int4*>(kinfo + 32 * k + x);
+        const int vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t u = uint32_t(vv[e]);
+          const bool in = ids ? (vv[e] == my_seg)
+                              : (uint32_t(int(u >> 22) - ws0) < uint32_t(k0) &&
+                                 uint32_t(int((u >> 11) & 2047u) - ws1) < uint32_t(k1) &&
+                                 uint32_t(int(u & 2047u) - ws2) < uint32_t(k2));
+          bits |= (in ? 1u : 0u) << (x + e);
+        }
+      }
+      mb[k] = bits;
+    }
+  }
+  uint32_t lim[4] = {0u, 0u, 0u, 0u};
+  set_bit_range(lim, 0, n_lim);
+  return make_uint4(mb[0] & lim[0], mb[1] & lim[1], mb[2] & lim[2], mb[3] & lim[3]);
+}
+
+// The same as a call, so that its registers do not weigh on the softmax's
+// where masked tiles are rare.
+__device__ __noinline__ uint4 tile_mask_call(const int32_t* kinfo, int mode, int my_seg, int ws0,
+                                             int ws1, int ws2, int k0, int k1, int k2,
+                                             int n_lim) {
+  return tile_mask(kinfo, mode, my_seg, ws0, ws1, ws2, k0, k1, k2, n_lim);
+}
+
 // One thread's row of a 128-column S tile from tensor memory.
 __device__ __forceinline__ void load_s_row(uint32_t taddr, float (&s)[kBN]) {
   uint32_t sr[4][32];
@@ -196,10 +378,11 @@ __device__ __forceinline__ float row_max(const float (&s)[kBN]) {
 // p = 2^(c*s - m) for a row of 128 scores: per 16 keys, the first 16 - kEmu
 // on the MUFU unit (ex2), the last kEmu on the FMA pipe (exp2_poly2).  The
 // bf16-rounded p go to pk (two per word, the layout of P in tensor memory);
-// returns the fp32 sum of p (four packed partial sums).
-template <int kEmu>
+// returns the fp32 sum of p (four packed partial sums).  kMasked: keys whose
+// bit in mb is clear get p = 0 (whatever their score).
+template <int kEmu, bool kMasked = false>
 __device__ __forceinline__ float exp_tile(const float (&s)[kBN], float c, float m,
-                                          uint32_t (&pk)[2][32]) {
+                                          uint32_t (&pk)[2][32], const uint32_t* mb = nullptr) {
   const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                    make_float2(0.f, 0.f)};
@@ -212,6 +395,10 @@ __device__ __forceinline__ float exp_tile(const float (&s)[kBN], float c, float 
       e.y = ex2(arg.y);
     } else {
       e = exp2_poly2(arg);
+    }
+    if constexpr (kMasked) {
+      e.x = ((mb[x >> 5] >> (x & 31)) & 1u) ? e.x : 0.f;
+      e.y = ((mb[x >> 5] >> ((x + 1) & 31)) & 1u) ? e.y : 0.f;
     }
     acc[(x >> 1) & 3] = fadd2(acc[(x >> 1) & 3], e);
     pk[x >> 6][(x >> 1) & 31] = pack_bf16x2(e.x, e.y);
@@ -254,10 +441,12 @@ __device__ __forceinline__ KvWalk make_walk(const FwdParams& p, int b, int pair,
   const int4* qsum_b = p.q_sum + static_cast<int64_t>(b) * p.n_q_tiles;
   const int4 q0 = __ldg(qsum_b + qt0);
   const int4 q1 = (qt0 + 1 < p.n_q_tiles) ? __ldg(qsum_b + qt0 + 1) : q0;
-  walk.kv_sum = p.kv_sum + static_cast<int64_t>(b) * p.n_kv_tiles;
-  walk.qmin = min(q0.x, q1.x);
-  walk.qmax = max(q0.y, q1.y);
   if (q_summary) *q_summary = (qi == 1) ? q1 : q0;
+  if (p.coord_q == nullptr) {   // ids: walk the tiles whose id range meets the queries'
+    walk.kv_sum = p.kv_sum + static_cast<int64_t>(b) * p.n_kv_tiles;
+    walk.qmin = min(q0.x, q1.x);
+    walk.qmax = max(q0.y, q1.y);
+  }
   return walk;
 }
 
@@ -303,7 +492,11 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 }
 
 // kEmu: exponentials per 16 keys computed on the FMA pipe instead of MUFU.
-template <int D, int kEmu>
+// kMaskFast: masked key tiles (D = 128) take the running-offset path with
+// their hidden keys' scores set to -inf, instead of the two-pass exact path
+// (the variant for 3D neighbourhood windows, where nearly every visited tile
+// is masked; elsewhere the extra code costs the unmasked tiles registers).
+template <int D, int kEmu, bool kMaskFast>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     vidattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -370,7 +563,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
 
-  const bool has_seg = p.q_sum != nullptr;
+  const bool has_sum = p.q_sum != nullptr;      // tile summaries: ids or window boxes
+  const bool has_win = p.coord_q != nullptr;
+  const bool has_seg = has_sum && !has_win;
   // key tiles visited end here (causal: past the last key any row sees)
   const int n_kv = causal_end(p, pair);
 #ifdef VIDATTN_TRACE
@@ -383,7 +578,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // touches global memory to find its next tile.
   int* tile_list = reinterpret_cast<int*>(smem + C::kOffList);
   int n_list = 0;
-  const bool listed = has_seg && n_kv <= kMaxListedTiles;
+  const bool listed = has_sum && n_kv <= kMaxListedTiles;
   if (listed) {
     int4 q0, q1;
     const KvWalk w = make_walk(p, b, pair, 0, &q0);
@@ -395,13 +590,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool act = false;
       int entry = 0;
       if (jj < n_kv) {
-        const int4 ks = __ldg(w.kv_sum + jj);
-        act = !(ks.y < w.qmin || ks.x > w.qmax);
+        const int4 ks = __ldg(p.kv_sum + static_cast<int64_t>(b) * p.n_kv_tiles + jj);
         const bool last_ragged = ragged && jj == p.n_kv_tiles - 1;
-        const bool m0 = last_ragged || !(q0.z && ks.z && q0.x == ks.x) ||
-                        causal_partial(p, pair, 0, jj);
-        const bool m1 = last_ragged || !(q1.z && ks.z && q1.x == ks.x) ||
-                        causal_partial(p, pair, 1, jj);
+        bool m0, m1;
+        if (has_win) {
+          act = win_tile_meets(p, q0, q1, ks);
+          m0 = last_ragged || !win_tile_full(p, q0, ks);
+          m1 = last_ragged || !win_tile_full(p, q1, ks);
+        } else {
+          act = !(ks.y < w.qmin || ks.x > w.qmax);
+          m0 = last_ragged || !(q0.z && ks.z && q0.x == ks.x) || causal_partial(p, pair, 0, jj);
+          m1 = last_ragged || !(q1.z && ks.z && q1.x == ks.x) || causal_partial(p, pair, 1, jj);
+        }
         entry = jj | (m0 ? (1 << 30) : 0) | (m1 ? int(1u << 31) : 0);
       }
       const unsigned ballot = __ballot_sync(0xffffffffu, act);
@@ -648,6 +848,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const bool row_valid = row < p.S_q;
     const int32_t* seg_kv_b = has_seg ? p.seg_kv + static_cast<int64_t>(b) * p.S_kv : nullptr;
     const int my_seg = (has_seg && row_valid) ? __ldg(p.seg_q + static_cast<int64_t>(b) * p.S_q + row) : 0;
+    const int32_t* coord_kv_b = has_win ? p.coord_kv + static_cast<int64_t>(b) * p.S_kv : nullptr;
+    const int32_t* coord_q_b = has_win ? p.coord_q + static_cast<int64_t>(b) * p.S_q : nullptr;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kTmemS + 128u * qi;
     const uint32_t tO = tmem + lane_off + C::kTmemO + uint32_t(D) * qi;
@@ -657,6 +859,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         make_walk(p, b, pair, qi, &my_qs)};
     const float c = p.c;
     const bool ragged_kv = (p.S_kv % kBN) != 0;
+    // masked key tiles: their keys' ids or coordinates, staged per warp
+    int32_t* kinfo = reinterpret_cast<int32_t*>(smem + C::kOffKinfo) + warp * kBN;
+    const int32_t* kinfo_src = has_win ? coord_kv_b : seg_kv_b;   // null with neither
+    const uint32_t my_coord = (has_win && row_valid) ? uint32_t(__ldg(coord_q_b + row)) : 0u;
 
     float m_run = -INFINITY;   // running max of scale*log2(e)*s, the offset of P
     float l_run = 0.f;         // running sum of P (fp32, before bf16 rounding)
@@ -667,18 +873,57 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (listed) {
         masked = (tile_list[t] >> (30 + qi)) & 1;
       } else {
-        masked = (ragged_kv && j == p.n_kv_tiles - 1) || causal_partial(p, pair, qi, j);
+        masked = (ragged_kv && j == p.n_kv_tiles - 1) || causal_partial(p, pair, qi, j) || has_win;
         if (has_seg) {
           const int4 ks = __ldg(sched.walk.kv_sum + j);
           masked = masked || !(my_qs.z && ks.z && my_qs.x == ks.x);
         }
       }
       const bool slow = masked || !(c > 0.f);
+      // A masked tile's key ids / coordinates: loads issued before the wait
+      // for S, so their latency hides behind it (warp-uniform: masked is the
+      // same for every row of a Q tile).
+      int32_t pre[4] = {0, 0, 0, 0};
+      if (masked && kinfo_src != nullptr) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int x = j * kBN + lane + 32 * m;
+          if (x < p.S_kv) pre[m] = __ldg(kinfo_src + x);
+        }
+      }
       VIDATTN_TR(1 + qi, t, 0);
       ok = warp_wait_phase(s_full(qi), t & 1, abort_flag, p.err);
       VIDATTN_TR(1 + qi, t, 1);
       if (!ok) break;
       tc_fence_after();
+      if (masked && kinfo_src != nullptr) {
+        // the previous masked tile's mask was built before this point (the
+        // __syncwarp after it), so the slot is free
+#pragma unroll
+        for (int m = 0; m < 4; ++m) kinfo[lane + 32 * m] = pre[m];
+      }
+      // visible keys of this row: all of an unmasked tile; a masked tile's
+      // mask is built where it is used (the exact paths), from the slot
+      auto build_mask = [&](uint32_t (&mb)[4]) {
+        const int j0 = j * kBN;
+        const int n_valid = min(kBN, p.S_kv - j0);
+        const int n_lim =
+            p.causal ? max(0, min(n_valid, row + p.causal_off - j0 + 1)) : n_valid;
+        const WinRow wr = win_row(p, my_coord);
+        __syncwarp();
+        const int mode = has_win ? 2 : (has_seg ? 1 : 0);
+        const uint4 m =
+            kMaskFast ? tile_mask(kinfo, mode, my_seg, wr.s[0], wr.s[1], wr.s[2], p.win_size[0],
+                                  p.win_size[1], p.win_size[2], n_lim)
+                      : tile_mask_call(kinfo, mode, my_seg, wr.s[0], wr.s[1], wr.s[2],
+                                       p.win_size[0], p.win_size[1], p.win_size[2], n_lim);
+        __syncwarp();   // every lane has read the slot before it is refilled
+        mb[0] = m.x;
+        mb[1] = m.y;
+        mb[2] = m.z;
+        mb[3] = m.w;
+      };
+
       if constexpr (C::kSepP) {
         // S row into registers, then S's columns are released to the MMA warp.
         float s[kBN];
@@ -701,12 +946,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (!slow) {
             tile_max = row_max(s) * c;
           } else {
-            const int j0 = j * kBN;
+            uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+            if (masked) build_mask(mb);
             float mx = -INFINITY;
 #pragma unroll
             for (int x = 0; x < kBN; ++x) {
-              bool valid = (j0 + x) < p.S_kv && (!p.causal || j0 + x <= row + p.causal_off);
-              if (has_seg && valid) valid = __ldg(seg_kv_b + j0 + x) == my_seg;
+              const bool valid = (mb[x >> 5] >> (x & 31)) & 1u;
               s[x] = valid ? s[x] * c : -INFINITY;
               mx = fmaxf(mx, s[x]);
             }
@@ -769,13 +1014,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // a row's first tile, and scale <= 0.
         float rs = 0.f, alpha = 1.f;
         bool rescale = false;
-        // warp-uniform choice: the stale path only if every row of the warp can take it
-        bool exact = __any_sync(0xffffffffu, slow || (m_run == -INFINITY));
+        // warp-uniform choice: the stale path only if every row of the warp
+        // can take it (with kMaskFast masked tiles too: hidden keys get p = 0)
+        bool exact = __any_sync(0xffffffffu, (kMaskFast ? !(c > 0.f) : slow) || (m_run == -INFINITY));
         if (!exact) {
+          // a masked tile: its mask first (before S occupies the registers),
+          // then hidden keys' scores become -inf, i.e. p = 0 (the FMA-pipe
+          // exponential clamps at 2^-125, far below bf16 P's resolution
+          // against the row sum, which includes the row's running maximum)
+          uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+          if (kMaskFast && masked) build_mask(mb);
           float s[kBN];
           uint32_t pk[2][32];
           load_s_row(tS, s);
           VIDATTN_TR(1 + qi, t, 2);
+          if (kMaskFast && masked) {
+#pragma unroll
+            for (int x = 0; x < kBN; ++x)
+              s[x] = ((mb[x >> 5] >> (x & 31)) & 1u) ? s[x] : -INFINITY;
+          }
           rs = exp_tile<kEmu>(s, c, m_run, pk);
           VIDATTN_TR(1 + qi, t, 3);
           exact = __any_sync(0xffffffffu, !(rs <= kStaleSumLimit));
@@ -789,22 +1046,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // tensor memory (S is intact: no P has been written yet).  The sum
           // restarts: a failed running-offset attempt leaves its sum in rs.
           rs = 0.f;
-          const int j0 = j * kBN;
-          auto allowed = [&](int x) {
-            bool valid = (j0 + x) < p.S_kv && (!p.causal || j0 + x <= row + p.causal_off);
-            if (has_seg && valid) valid = __ldg(seg_kv_b + j0 + x) == my_seg;
-            return valid;
+          uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+          if (masked) build_mask(mb);
+          // this chunk's 32 mask bits (k is a runtime index: select, don't index)
+          auto chunk_bits = [&](int k) {
+            return k == 0 ? mb[0] : (k == 1 ? mb[1] : (k == 2 ? mb[2] : mb[3]));
           };
           float mx = -INFINITY;
   #pragma unroll 1
           for (int k = 0; k < 4; ++k) {
             uint32_t r[32];
             tmem_ld32(tS + 32 * k, r);
+            const uint32_t mk = chunk_bits(k);
             tmem_ld_wait();
             reg_fence(r);
   #pragma unroll
             for (int x = 0; x < 32; ++x)
-              mx = fmaxf(mx, allowed(32 * k + x) ? __uint_as_float(r[x]) * c : -INFINITY);
+              mx = fmaxf(mx, ((mk >> x) & 1u) ? __uint_as_float(r[x]) * c : -INFINITY);
           }
           const float m_new = fmaxf(m_run, mx);
           rescale = (m_new - m_run) > kRescaleThreshold;   // false for -inf - -inf
@@ -819,13 +1077,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int k = 0; k < 4; ++k) {
             uint32_t r[32], w[16];
             tmem_ld32(tS + 32 * k, r);
+            const uint32_t mk = chunk_bits(k);
             tmem_ld_wait();
             reg_fence(r);
   #pragma unroll
             for (int x = 0; x < 32; x += 2) {
-              const float e0 = allowed(32 * k + x) ? ex2(__uint_as_float(r[x]) * c - msub) : 0.f;
+              const float e0 = ((mk >> x) & 1u) ? ex2(__uint_as_float(r[x]) * c - msub) : 0.f;
               const float e1 =
-                  allowed(32 * k + x + 1) ? ex2(__uint_as_float(r[x + 1]) * c - msub) : 0.f;
+                  ((mk >> (x + 1)) & 1u) ? ex2(__uint_as_float(r[x + 1]) * c - msub) : 0.f;
               rs += e0 + e1;
               w[x >> 1] = pack_bf16x2(e0, e1);
             }

@@ -110,12 +110,17 @@ constexpr int kNumEmu = 5;
 template <int D>
 FwdKernel fwd_variant(int e) {
   switch (e) {
-    case 0: return vidattn_fwd_kernel<D, 0>;
-    case 1: return vidattn_fwd_kernel<D, 2>;
-    case 2: return vidattn_fwd_kernel<D, 4>;
-    case 3: return vidattn_fwd_kernel<D, 6>;
-    default: return vidattn_fwd_kernel<D, 8>;
+    case 0: return vidattn_fwd_kernel<D, 0, false>;
+    case 1: return vidattn_fwd_kernel<D, 2, false>;
+    case 2: return vidattn_fwd_kernel<D, 4, false>;
+    case 3: return vidattn_fwd_kernel<D, 6, false>;
+    default: return vidattn_fwd_kernel<D, 8, false>;
   }
+}
+// 3D neighbourhood windows: masked tiles on the running-offset path (D = 128,
+// the default 4 of 16 exponentials on the FMA pipe); D = 64 uses the default.
+FwdKernel fwd_window_variant(int D) {
+  return D == 128 ? vidattn_fwd_kernel<128, 4, true> : vidattn_fwd_kernel<64, 2, false>;
 }
 // Default share of exponentials moved off the MUFU unit (measured best on
 // B200: 4 of 16 at D = 128, 2 of 16 at D = 64, where the FMA-pipe version's
@@ -171,6 +176,9 @@ int ensure_device(int* dev_out) {
                                FwdCfg<128>::kSmemBytes) != cudaSuccess)
         return VIDATTN_ERR_CUDA;
     }
+    if (cudaFuncSetAttribute(fwd_window_variant(128), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FwdCfg<128>::kSmemBytes) != cudaSuccess)
+      return VIDATTN_ERR_CUDA;
     info.attrs_set = 1;
   }
   return VIDATTN_OK;
@@ -261,11 +269,18 @@ int check_args(const void* q, const void* k, const void* v, const int32_t* seg_q
   return VIDATTN_OK;
 }
 
+// A 3D neighbourhood window for launch_fwd.
+struct WinSpec {
+  const int32_t* coord_q;
+  const int32_t* coord_kv;
+  int size[3], extent[3], clamped;
+};
+
 template <int D>
 int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32_t* seg_q,
                const int32_t* seg_kv, const int4* q_sum, const int4* kv_sum, void* out,
                float* lse, int B, int H, int S_q, int S_kv, float scale, cudaStream_t stream,
-               int flags = 0) {
+               int flags = 0, const WinSpec* win = nullptr) {
   CUtensorMap tq, tk, tv;
   const int64_t BH = int64_t(B) * H;
   // With no keys the K/V maps are never read; they are encoded over q.
@@ -289,12 +304,21 @@ int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32
   p.n_kv_tiles = (S_kv + kBN - 1) / kBN;
   p.causal = (flags & VIDATTN_CAUSAL) ? 1 : 0;
   p.causal_off = S_kv - S_q;
+  if (win) {
+    p.coord_q = win->coord_q;
+    p.coord_kv = win->coord_kv;
+    for (int a = 0; a < 3; ++a) {
+      p.win_size[a] = win->size[a];
+      p.win_extent[a] = win->extent[a];
+    }
+    p.win_clamped = win->clamped;
+  }
   p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
 #ifdef VIDATTN_TRACE
   p.trace = g_trace;
 #endif
   dim3 grid((S_q + 2 * kBM - 1) / (2 * kBM), H, B);
-  FwdKernel kernel = fwd_variant<D>(emu_index(D));
+  FwdKernel kernel = win ? fwd_window_variant(D) : fwd_variant<D>(emu_index(D));
   kernel<<<grid, kFwdThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? VIDATTN_OK : VIDATTN_ERR_CUDA;
 }
@@ -437,6 +461,49 @@ VIDATTN_API int vidattn_fwd_ex(const void* q, const void* k, const void* v,
                           stream, flags);
   return launch_fwd<128>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
                          stream, flags);
+}
+
+VIDATTN_API int vidattn_fwd_window(const void* q, const void* k, const void* v,
+                                   const int32_t* coord_q, const int32_t* coord_kv, void* out,
+                                   float* lse, int B, int H, int S_q, int S_kv, int D,
+                                   float scale, int win_t, int win_h, int win_w, int T, int Hg,
+                                   int Wg, int flags, vidattn_stream_t stream_) {
+  if (!coord_q || !coord_kv) return VIDATTN_ERR_NULL;
+  if (flags & ~VIDATTN_WINDOW_CLAMPED) return VIDATTN_ERR_BAD_SHAPE;
+  int st = check_args(q, k, v, coord_q, coord_kv, out, lse, B, H, S_q, S_kv, D);
+  if (st != VIDATTN_OK) return st;
+  if (!std::isfinite(scale)) return VIDATTN_ERR_BAD_SHAPE;
+  const int size[3] = {win_t, win_h, win_w};
+  const int extent[3] = {T, Hg, Wg};
+  const int max_extent[3] = {1024, 2048, 2048};
+  for (int a = 0; a < 3; ++a) {
+    if (size[a] < 1 || size[a] % 2 == 0 || extent[a] < 1 || extent[a] > max_extent[a])
+      return VIDATTN_ERR_BAD_SHAPE;
+  }
+  if (int64_t(S_kv) > int64_t(kMaxListedTiles) * kBN) return VIDATTN_ERR_BAD_SHAPE;
+  if (S_q == 0) return VIDATTN_OK;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int dev = 0;
+  st = ensure_device(&dev);
+  if (st != VIDATTN_OK) return st;
+
+  const int nq = (S_q + kSegTile - 1) / kSegTile;
+  const int nk = (S_kv + kSegTile - 1) / kSegTile;
+  const size_t bytes = sizeof(int4) * size_t(B) * (size_t(nq) + size_t(nk > 0 ? nk : 1));
+  int4* buf = static_cast<int4*>(scratch_for(dev, stream, bytes));
+  if (!buf) return VIDATTN_ERR_CUDA;
+  int4* q_box = buf;
+  int4* kv_box = buf + size_t(B) * nq;
+  dim3 grid(nq > nk ? nq : nk, B, 2);
+  win_tile_bbox_kernel<<<grid, 128, 0, stream>>>(coord_q, coord_kv, q_box, kv_box, S_q, S_kv);
+  if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
+  WinSpec win{coord_q, coord_kv, {win_t, win_h, win_w}, {T, Hg, Wg},
+              (flags & VIDATTN_WINDOW_CLAMPED) ? 1 : 0};
+  if (D == 64)
+    return launch_fwd<64>(dev, q, k, v, nullptr, nullptr, q_box, kv_box, out, lse, B, H, S_q, S_kv,
+                          scale, stream, 0, &win);
+  return launch_fwd<128>(dev, q, k, v, nullptr, nullptr, q_box, kv_box, out, lse, B, H, S_q, S_kv,
+                         scale, stream, 0, &win);
 }
 
 VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h_v,

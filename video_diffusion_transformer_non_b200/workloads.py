@@ -15,12 +15,18 @@ Recipe (every tensor is seeded; nothing is loaded from disk):
   see bit-identical inputs;
 * segment ids are int32 [B, S]: contiguous runs in the order video, text, pad.
 
-The five named workloads follow the token counts of the video latents in the
+The first five named workloads follow the token counts of the video latents in the
 paper's benchmark families (vidax: A Unified JAX Framework for Video Generative
 Models on Accelerator Meshes, Fig. 1 and Tables 2 and 5: 480p and 720p
 Wan/HunyuanVideo grids, CogVideoX 720x480x49 with a 226-token T5 prompt), and
 stand in for them; the head counts and head dims are those of the named DiT
 families.
+
+The two window workloads stand in for the 3D neighbourhood attention of the
+LTX-2.5 VAE decoder (same paper, Appendix A, Table 4, group 4: an 11 x 11 x 11
+window); the paper gives neither its volume nor its heads, so window_480p
+runs that window over the 480p latent volume with 16 heads of 128, and
+window_small is the quick case.  Their tokens are the volume in raster order.
 
 The rotary-embedding conventions attached to each workload (the paper names
 3D RoPE per family but prints none) are taken from the families' public
@@ -56,6 +62,10 @@ class Workload:
     rope_bands: tuple | None = None
     rope_theta: float = 10000.0
     rope_interleaved: bool = True
+    # 3D neighbourhood attention over the rope_grid volume (all S tokens are
+    # video tokens in raster order): odd window size per axis, clamped or not
+    window: tuple | None = None
+    window_clamped: bool = True
 
     @property
     def S_q(self) -> int:
@@ -99,11 +109,72 @@ WORKLOADS = {
         segments=((118800, 0), (256, 1), (112, 2)), S=119168, seed=4,
         description="B1 H24 D128: 118800 video (33x45x80) + 256 text + 112 pad; ids video 0, text 1, pad 2",
         rope_grid=(33, 45, 80), rope_bands=(16, 56, 56), rope_theta=256.0),
+    "window_small": Workload(
+        name="window_small", B=2, H=4, D=128, segments=None, S=2048, seed=5,
+        description="B2 H4 D128: 3D neighbourhood attention over an 8x16x16 volume, "
+                    "window 5x5x5 clamped",
+        rope_grid=(8, 16, 16), rope_bands=(44, 42, 42), window=(5, 5, 5)),
+    "window_480p": Workload(
+        name="window_480p", B=1, H=16, D=128, segments=None, S=32760, seed=6,
+        description="B1 H16 D128: 3D neighbourhood attention over the 21x30x52 latent volume, "
+                    "window 11x11x11 clamped",
+        rope_grid=(21, 30, 52), rope_bands=(44, 42, 42), window=(11, 11, 11)),
 }
 
 for _w in WORKLOADS.values():
     assert _w.segments is None or _runs_total(_w.segments) == _w.S, _w.name
     assert _w.rope_offset + int(np.prod(_w.rope_grid)) <= _w.S and sum(_w.rope_bands) == _w.D, _w.name
+
+
+def pack_coords(t, h, w) -> np.ndarray:
+    """Per-token coordinates packed t << 22 | h << 11 | w, as int32."""
+    return ((np.asarray(t, np.int64) << 22) | (np.asarray(h, np.int64) << 11)
+            | np.asarray(w, np.int64)).astype(np.uint32).view(np.int32)
+
+
+def raster_coords(grid, B: int) -> np.ndarray:
+    """int32 [B, T*Hg*Wg]: the packed (t, h, w) of each token of a T x Hg x Wg
+    volume in raster order (w fastest), the same for every sample."""
+    T, Hg, Wg = grid
+    t, h, w = np.meshgrid(np.arange(T), np.arange(Hg), np.arange(Wg), indexing="ij")
+    c = pack_coords(t.ravel(), h.ravel(), w.ravel())
+    return np.ascontiguousarray(np.broadcast_to(c, (B, c.size)))
+
+
+def window_of(w: Workload, B: int | None = None) -> dict:
+    """The window description of a windowed workload (oracle and binding form)."""
+    c = raster_coords(w.rope_grid, w.B if B is None else B)
+    return dict(coord_q=c, coord_kv=c.copy(), size=w.window, extent=w.rope_grid,
+                clamped=w.window_clamped)
+
+
+def window_pairs(w: Workload) -> int:
+    """(query, key) pairs inside the windows over the whole volume, per sample
+    and head: the per-axis counts multiply, so the total is the product over
+    axes of the sum over coordinates of the window length on that axis."""
+    total = 1
+    for k, N in zip(w.window, w.rope_grid):
+        r = (k - 1) // 2
+        c = np.arange(N)
+        if w.window_clamped:
+            per = np.full(N, min(k, N))
+        else:
+            per = np.minimum(c + r, N - 1) - np.maximum(c - r, 0) + 1
+        total *= int(per.sum())
+    return total
+
+
+def window_row_counts(w: Workload, rows) -> np.ndarray:
+    """Keys inside the window of each query row (sequence index, raster order)."""
+    T, Hg, Wg = w.rope_grid
+    rows = np.asarray(rows, np.int64)
+    coords = (rows // (Hg * Wg), (rows // Wg) % Hg, rows % Wg)
+    n = np.ones(rows.shape, np.int64)
+    for c, k, N in zip(coords, w.window, w.rope_grid):
+        r = (k - 1) // 2
+        n *= (np.full(c.shape, min(k, N)) if w.window_clamped
+              else np.minimum(c + r, N - 1) - np.maximum(c - r, 0) + 1)
+    return n
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -173,6 +244,8 @@ def allowed_pairs(w_or_seg_q, seg_kv=None, S_q=None, S_kv=None, B=None) -> int:
     Counted from the runs, without building any mask."""
     if isinstance(w_or_seg_q, Workload):
         w = w_or_seg_q
+        if w.window is not None:
+            return w.B * window_pairs(w)
         if w.segments is None:
             return w.B * w.S_q * w.S_kv
         per_id = {}
