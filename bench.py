@@ -50,14 +50,16 @@ def load_peaks():
 
 
 KERNEL_SOURCES = ["fwd_kernel.cuh", "ptx.cuh", "vidattn.cu", "classify.cuh"]
+ROPE_SOURCES = ["rope3d.cuh", "ptx.cuh", "vidattn.cu"]
 
 
-def measured_traffic(w):
+def measured_traffic(w, summary=None, sources=KERNEL_SOURCES):
     """DRAM bytes per launch from the committed ncu summary of this workload's
     kernel, or None when there is none or the kernel sources changed since."""
     import hashlib
     import re
-    path = os.path.join(ROOT, "profiles", f"vidattn_fwd_kernel_d{w.D}__{w.name}_h8.md")
+    path = os.path.join(ROOT, "profiles",
+                        summary or f"vidattn_fwd_kernel_d{w.D}__{w.name}_h8.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -67,7 +69,7 @@ def measured_traffic(w):
         return None
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "video_diffusion_transformer_non_b200", "csrc")
-    for f in KERNEL_SOURCES:
+    for f in sources:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return int(val.group(1)) if h.hexdigest() == sha.group(1) else None
@@ -491,7 +493,10 @@ def main(argv=None):
                                "pairing": "interleaved" if rope_interleaved else "half-split"},
                 "roofline": {"bound": "hbm", "achieved": r_gbs, "peak": peaks["hbm"],
                              "unit": "GB/s", "frac": r_gbs / peaks["hbm"],
-                             "traffic": None, "peak_source": f"{peaks['source']} HBM copy",
+                             "traffic": (measured_traffic(
+                                 w, f"rope3d_kernel_d{w.D}__{w.name}.md", ROPE_SOURCES)
+                                 if rope_interleaved and args.heads is None else None),
+                             "peak_source": f"{peaks['source']} HBM copy",
                              "algorithmic_bytes_per_launch": r_bytes}}
 
     cpu = None

@@ -10,10 +10,11 @@
 //
 // Work split: a tile is kRopeTokens consecutive tokens of every (tensor, b, h)
 // slab.  The CTA computes the tile's (cos, sin) table once in shared memory
-// (the angles in fp64, reduced to [-pi, pi], then sincosf), each thread keeps
-// the entries of its own 8 features in registers and then streams 16-byte
-// chunks of all slabs through them: kRopeUnroll loads in flight per thread,
-// streaming-cache loads and stores (every byte is touched once).  The
+// (the angles in fp64, reduced to [-pi, pi], then sincosf; two tables
+// alternate, so one barrier per tile suffices), each thread keeps the entries
+// of its own 8 features in registers and then streams 16-byte chunks of all
+// slabs through them: kRopeUnroll loads in flight per thread, streaming-cache
+// loads and stores (every byte is touched once).  The
 // interleaved pairing finds both features of a pair in one chunk; the
 // half-split pairing stages the chunk in shared memory and reads the partner
 // feature from the neighbouring thread of the same row.
@@ -27,7 +28,7 @@
 namespace vidattn {
 
 constexpr int kRopeThreads = 256;
-constexpr int kRopeTokens = 4;
+constexpr int kRopeTokens = 8;
 constexpr int kRopeUnroll = 4;
 constexpr int kRopeMaxD = 128;
 
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __grid_const
   constexpr int kSlabsPerPass = kRopeThreads / kPerSlab;
   static_assert(kRopeThreads % kPerSlab == 0 && 32 % kChunks == 0, "tile shape");
 
-  __shared__ float2 table[kRopeTokens][kHalf];
+  __shared__ __align__(16) float2 table[2][kRopeTokens][kHalf];
   __shared__ uint4 stage[kInterleaved ? 1 : kRopeUnroll][kRopeThreads];
 
   const int tid = threadIdx.x;
@@ -101,9 +102,12 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __grid_const
     partner_elem[e] = p.partner[f] % 8;
   }
 
-  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+  int parity = 0;
+  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, parity ^= 1) {
     const int s0 = tile * kRopeTokens;
-    __syncthreads();  // the previous tile's table is no longer read
+    // this tile's table goes to the buffer read two tiles ago: every thread
+    // has passed the previous tile's barrier, so it is done reading it
+    float2 (*tb)[kHalf] = table[parity];
     for (int i = tid; i < kRopeTokens * kHalf; i += kRopeThreads) {
       const int r = i / kHalf, c = i % kHalf;
       const int n = s0 + r - p.offset;
@@ -115,16 +119,28 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __grid_const
         a -= two_pi * rint(a / two_pi);
         sincosf(float(a), &sv, &cv);
       }
-      table[r][c] = make_float2(cv, sv);
+      tb[r][c] = make_float2(cv, sv);
     }
     __syncthreads();
 
     float cs[8], sn[8];
+    if constexpr (kInterleaved) {
+      // features 8ch .. 8ch+7 are the pairs (columns) 4ch .. 4ch+3
+      const float4 a = *reinterpret_cast<const float4*>(&tb[row][4 * ch]);
+      const float4 b = *reinterpret_cast<const float4*>(&tb[row][4 * ch + 2]);
+      const float cc[4] = {a.x, a.z, b.x, b.z}, ss[4] = {a.y, a.w, b.y, b.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float2 t = table[row][col[e]];
-      cs[e] = t.x;
-      sn[e] = first[e] ? -t.y : t.y;
+      for (int e = 0; e < 8; ++e) {
+        cs[e] = cc[e >> 1];
+        sn[e] = (e & 1) ? ss[e >> 1] : -ss[e >> 1];
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float2 t = tb[row][col[e]];
+        cs[e] = t.x;
+        sn[e] = first[e] ? -t.y : t.y;
+      }
     }
     const int s = s0 + row;
     const bool row_ok = s < p.S;
