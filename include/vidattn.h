@@ -172,10 +172,18 @@ VIDATTN_API int vidattn_fwd_window(const void* q, const void* k, const void* v,
  * data lives in host memory.  h_* are host pointers (pinned memory gives
  * asynchronous copies; pageable memory works but the copies then block);
  * d_* are caller-owned device staging buffers of the same shapes, with the
- * alignment rules of vidattn_fwd.  Enqueued on `stream`, in order: one
- * host-to-device copy per input (q, k, v, then seg_q, seg_kv when given), the
- * forward, then device-to-host copies of out and lse.  The host outputs are
- * valid once the stream has been synchronised.  h_seg_q/h_seg_kv and
+ * alignment rules of vidattn_fwd.  Enqueued behind the work already on
+ * `stream`: the ids (when given) are copied in on `stream`; then, for small
+ * problems (under 64 MiB of copies, or H = 1), q, k, v are copied in, the
+ * forward runs and out, lse are copied back, all on `stream`.  Larger
+ * problems are pipelined over chunks of heads (up to 4 per batch entry):
+ * chunk c+1's inputs are copied in and chunk c-1's outputs copied back, on
+ * two copy streams the library keeps per device (created on first use,
+ * destroyed by vidattn_release), while chunk c's forward runs on `stream`;
+ * events order the three steps of each chunk, and `stream` waits for the
+ * last copy.  Either way the host outputs are valid once `stream` has been
+ * synchronised, and they equal vidattn_fwd's bit for bit.  Host buffers
+ * should be pinned for the copies to overlap.  h_seg_q/h_seg_kv and
  * d_seg_q/d_seg_kv follow the NULL rule of vidattn_fwd.
  */
 VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h_v,

@@ -189,6 +189,42 @@ def test_host_buffer_entry_point_matches_device_entry_point():
     assert torch.equal(hlse, lse_d.cpu())
 
 
+@pytest.mark.parametrize("with_ids,S_q,S_kv", [(True, 8192, 8192), (False, 6000, 9000)])
+def test_pipelined_host_entry_point_matches_device_entry_point(with_ids, S_q, S_kv):
+    """Over 64 MiB of copies: vidattn_fwd_host pipelines chunks of heads
+    (B = 2, H = 5: chunks of 2, 2 and 1 heads per batch entry) across its
+    copy streams; the outputs equal the device entry point's bit for bit."""
+    B, H, D = 2, 5, 128
+    seg_q = seg_kv = None
+    if with_ids:
+        seg_q = np.zeros((B, S_q), np.int32)
+        seg_q[:, S_q - 300:] = 1
+        seg_q[1, :1000] = 2
+        seg_kv = seg_q.copy()
+    c = wl.make_random(B, H, S_q, S_kv, D, 44, seg_q, seg_kv)
+    out_d, lse_d = run_gpu(c, check=False)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    hq, hk, hv = (pin(c[n].view(np.int16)) for n in ("q", "k", "v"))
+    hsq = hsk = dsq = dsk = None
+    if with_ids:
+        hsq, hsk = pin(c["seg_q"]), pin(c["seg_kv"])
+        dsq = torch.empty((B, S_q), dtype=torch.int32, device="cuda")
+        dsk = torch.empty((B, S_kv), dtype=torch.int32, device="cuda")
+    hout = torch.empty((B, H, S_q, D), dtype=torch.int16).pin_memory()
+    hlse = torch.empty((B, H, S_q), dtype=torch.float32).pin_memory()
+    dq = torch.empty((B, H, S_q, D), dtype=torch.bfloat16, device="cuda")
+    dk, dv = (torch.empty((B, H, S_kv, D), dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    dout = torch.empty_like(dq)
+    dlse = torch.empty((B, H, S_q), dtype=torch.float32, device="cuda")
+    st = binding.vidattn_fwd_host(hq, hk, hv, hsq, hsk, hout, hlse, dq, dk, dv, dsq, dsk,
+                                  dout, dlse, B, H, S_q, S_kv, D, c["scale"])
+    assert st == 0
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    assert torch.equal(hout, out_d.view(torch.int16).cpu())
+    assert torch.equal(hlse, lse_d.cpu())
+
+
 def test_kernel_wait_timeout_is_reported_not_hung():
     """A kernel whose barrier never completes gives up after its time limit and
     reports through the device error word; the context stays usable."""

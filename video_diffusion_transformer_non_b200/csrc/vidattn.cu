@@ -77,6 +77,8 @@ struct DeviceInfo {
   uint32_t attrs_set = 0;   // bit (kernel variant index) once its smem limit is raised
   int* err = nullptr;       // device address of g_device_error on this device
   int rope_grid[4] = {};    // persistent grid of each rope3d variant (SMs x resident CTAs)
+  // vidattn_fwd_host's copy streams (host-to-device, device-to-host)
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
 };
 
 // Recently encoded tensor maps (per device): a call on the same buffers and
@@ -323,6 +325,25 @@ int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32
   return cudaGetLastError() == cudaSuccess ? VIDATTN_OK : VIDATTN_ERR_CUDA;
 }
 
+// The copy streams of vidattn_fwd_host on device dev (created on first use).
+bool copy_streams(int dev, cudaStream_t* in, cudaStream_t* out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& info = g_devices[dev];
+  if (!info.copy_in &&
+      cudaStreamCreateWithFlags(&info.copy_in, cudaStreamNonBlocking) != cudaSuccess)
+    return false;
+  if (!info.copy_out &&
+      cudaStreamCreateWithFlags(&info.copy_out, cudaStreamNonBlocking) != cudaSuccess)
+    return false;
+  *in = info.copy_in;
+  *out = info.copy_out;
+  return true;
+}
+
+// Below this many bytes of copies, vidattn_fwd_host does not split the work.
+constexpr size_t kPipelineMinBytes = size_t(64) << 20;
+constexpr int kPipelineChunks = 4;
+
 // One warp waits on an mbarrier that nothing ever arrives on, through the
 // attention kernel's bounded wait; it gives up after timeout_ns and reports.
 __global__ void selftest_timeout_kernel(int* err, unsigned long long timeout_ns) {
@@ -528,15 +549,83 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
   auto d2h = [&](void* h, const void* d, size_t n) {
     return n == 0 || cudaMemcpyAsync(h, d, n, cudaMemcpyDeviceToHost, stream) == cudaSuccess;
   };
-  if (!h2d(d_q, h_q, qb) || !h2d(d_k, h_k, kvb) || !h2d(d_v, h_v, kvb)) return VIDATTN_ERR_CUDA;
+  if (S_q == 0) return VIDATTN_OK;
   if (h_seg_q && (!h2d(d_seg_q, h_seg_q, size_t(B) * S_q * 4) ||
                   !h2d(d_seg_kv, h_seg_kv, size_t(B) * S_kv * 4)))
     return VIDATTN_ERR_CUDA;
-  st = vidattn_fwd(d_q, d_k, d_v, d_seg_q, d_seg_kv, d_out, d_lse, B, H, S_q, S_kv, D, scale,
-                   stream_);
+  const size_t lseb = size_t(B) * H * S_q * 4;
+  if (2 * qb + 2 * kvb < kPipelineMinBytes || H < 2) {
+    if (!h2d(d_q, h_q, qb) || !h2d(d_k, h_k, kvb) || !h2d(d_v, h_v, kvb)) return VIDATTN_ERR_CUDA;
+    st = vidattn_fwd(d_q, d_k, d_v, d_seg_q, d_seg_kv, d_out, d_lse, B, H, S_q, S_kv, D, scale,
+                     stream_);
+    if (st != VIDATTN_OK) return st;
+    if (!d2h(h_out, d_out, qb) || !d2h(h_lse, d_lse, lseb)) return VIDATTN_ERR_CUDA;
+    return VIDATTN_OK;
+  }
+
+  // Pipelined by chunks of heads: the copy-in of chunk c+1 and the copy-out
+  // of chunk c-1 run on two copy streams while chunk c's attention runs on
+  // `stream`; events order each chunk's copy-in, attention and copy-out.
+  // The heads are independent, so the result is the same, bit for bit.
+  int dev = 0;
+  st = ensure_device(&dev);
   if (st != VIDATTN_OK) return st;
-  if (!d2h(h_out, d_out, qb) || !d2h(h_lse, d_lse, size_t(B) * H * S_q * 4))
-    return VIDATTN_ERR_CUDA;
+  cudaStream_t cin = nullptr, cout = nullptr;
+  if (!copy_streams(dev, &cin, &cout)) return VIDATTN_ERR_CUDA;
+  const int hc = (H + kPipelineChunks - 1) / kPipelineChunks;
+  const size_t hq = size_t(S_q) * D * 2, hkv = size_t(S_kv) * D * 2, hl = size_t(S_q) * 4;
+  auto ev = [](cudaEvent_t* e) {
+    return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+  };
+  cudaEvent_t start, done;
+  if (!ev(&start) || !ev(&done)) return VIDATTN_ERR_CUDA;
+  bool ok = cudaEventRecord(start, stream) == cudaSuccess &&
+            cudaStreamWaitEvent(cin, start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(cout, start, 0) == cudaSuccess;
+  auto* cq = static_cast<const char*>(h_q);
+  auto* ck = static_cast<const char*>(h_k);
+  auto* cv = static_cast<const char*>(h_v);
+  for (int b = 0; ok && b < B; ++b) {
+    for (int h0 = 0; ok && h0 < H; h0 += hc) {
+      const int nh = (H - h0) < hc ? (H - h0) : hc;
+      const size_t u = size_t(b) * H + h0;   // first (b, h) slab of the chunk
+      char* dq = static_cast<char*>(d_q) + u * hq;
+      char* dk = static_cast<char*>(d_k) + u * hkv;
+      char* dv = static_cast<char*>(d_v) + u * hkv;
+      char* dout = static_cast<char*>(d_out) + u * hq;
+      float* dl = d_lse + u * S_q;
+      cudaEvent_t in_done, k_done;
+      if (!ev(&in_done) || !ev(&k_done)) return VIDATTN_ERR_CUDA;
+      ok = cudaMemcpyAsync(dq, cq + u * hq, nh * hq, cudaMemcpyHostToDevice, cin) == cudaSuccess &&
+           (S_kv == 0 ||
+            (cudaMemcpyAsync(dk, ck + u * hkv, nh * hkv, cudaMemcpyHostToDevice, cin) ==
+                 cudaSuccess &&
+             cudaMemcpyAsync(dv, cv + u * hkv, nh * hkv, cudaMemcpyHostToDevice, cin) ==
+                 cudaSuccess)) &&
+           cudaEventRecord(in_done, cin) == cudaSuccess &&
+           cudaStreamWaitEvent(stream, in_done, 0) == cudaSuccess;
+      if (ok) {
+        st = vidattn_fwd(dq, dk, dv, d_seg_q ? d_seg_q + size_t(b) * S_q : nullptr,
+                         d_seg_kv ? d_seg_kv + size_t(b) * S_kv : nullptr, dout, dl, 1, nh, S_q,
+                         S_kv, D, scale, stream_);
+        ok = st == VIDATTN_OK;
+      }
+      ok = ok && cudaEventRecord(k_done, stream) == cudaSuccess &&
+           cudaStreamWaitEvent(cout, k_done, 0) == cudaSuccess &&
+           cudaMemcpyAsync(static_cast<char*>(h_out) + u * hq, dout, nh * hq,
+                           cudaMemcpyDeviceToHost, cout) == cudaSuccess &&
+           cudaMemcpyAsync(h_lse + u * S_q, dl, nh * hl, cudaMemcpyDeviceToHost, cout) ==
+               cudaSuccess;
+      cudaEventDestroy(in_done);   // released once complete
+      cudaEventDestroy(k_done);
+    }
+  }
+  // `stream` reaches this point only after the last copy-out
+  ok = ok && cudaEventRecord(done, cout) == cudaSuccess &&
+       cudaStreamWaitEvent(stream, done, 0) == cudaSuccess;
+  cudaEventDestroy(start);
+  cudaEventDestroy(done);
+  if (!ok) return st != VIDATTN_OK ? st : VIDATTN_ERR_CUDA;
   return VIDATTN_OK;
 }
 
@@ -671,9 +760,25 @@ VIDATTN_API int vidattn_selftest_timeout(int timeout_us, vidattn_stream_t stream
 
 VIDATTN_API void vidattn_release(void) {
   std::lock_guard<std::mutex> lk(g_mu);
-  if (g_scratch.empty()) return;
   int prev = 0;
   cudaGetDevice(&prev);
+  for (auto& kv : g_devices) {
+    DeviceInfo& info = kv.second;
+    if (info.copy_in || info.copy_out) {
+      cudaSetDevice(kv.first);
+      for (cudaStream_t* sp : {&info.copy_in, &info.copy_out}) {
+        if (*sp) {
+          cudaStreamSynchronize(*sp);
+          cudaStreamDestroy(*sp);
+          *sp = nullptr;
+        }
+      }
+    }
+  }
+  if (g_scratch.empty()) {
+    cudaSetDevice(prev);
+    return;
+  }
   for (auto& kv : g_scratch) {
     if (kv.second.ptr) {
       cudaSetDevice(kv.first.first);
