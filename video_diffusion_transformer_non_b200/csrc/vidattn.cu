@@ -577,8 +577,11 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
   auto ev = [](cudaEvent_t* e) {
     return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
   };
-  cudaEvent_t start, done;
-  if (!ev(&start) || !ev(&done)) return VIDATTN_ERR_CUDA;
+  cudaEvent_t start = nullptr, done = nullptr;
+  if (!ev(&start) || !ev(&done)) {
+    if (start) cudaEventDestroy(start);
+    return VIDATTN_ERR_CUDA;
+  }
   bool ok = cudaEventRecord(start, stream) == cudaSuccess &&
             cudaStreamWaitEvent(cin, start, 0) == cudaSuccess &&
             cudaStreamWaitEvent(cout, start, 0) == cudaSuccess;
@@ -594,8 +597,12 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
       char* dv = static_cast<char*>(d_v) + u * hkv;
       char* dout = static_cast<char*>(d_out) + u * hq;
       float* dl = d_lse + u * S_q;
-      cudaEvent_t in_done, k_done;
-      if (!ev(&in_done) || !ev(&k_done)) return VIDATTN_ERR_CUDA;
+      cudaEvent_t in_done = nullptr, k_done = nullptr;
+      if (!ev(&in_done) || !ev(&k_done)) {
+        if (in_done) cudaEventDestroy(in_done);
+        ok = false;
+        break;
+      }
       ok = cudaMemcpyAsync(dq, cq + u * hq, nh * hq, cudaMemcpyHostToDevice, cin) == cudaSuccess &&
            (S_kv == 0 ||
             (cudaMemcpyAsync(dk, ck + u * hkv, nh * hkv, cudaMemcpyHostToDevice, cin) ==
