@@ -411,7 +411,7 @@ def main(argv=None):
     # forward, out and lse copied back, every step
     e2e = None
     if not args.no_e2e:
-        pin = lambda a: torch.from_numpy(a).pin_memory()
+        pin = lambda a: torch.from_numpy(a if a.flags.writeable else a.copy()).pin_memory()
         hq, hk, hv = (pin(inputs[n].view(np.int16)) for n in ("q", "k", "v"))
         hsq = None if inputs["seg_q"] is None else pin(inputs["seg_q"])
         hsk = None if inputs["seg_kv"] is None else pin(inputs["seg_kv"])

@@ -176,12 +176,12 @@ VIDATTN_API int vidattn_fwd_window(const void* q, const void* k, const void* v,
  * `stream`: the ids (when given) are copied in on `stream`; then, for small
  * problems (under 64 MiB of copies, or H = 1), q, k, v are copied in, the
  * forward runs and out, lse are copied back, all on `stream`.  Larger
- * problems are pipelined over chunks of heads (up to 4 per batch entry):
+ * problems are pipelined over chunks of heads (up to 8 per batch entry):
  * chunk c+1's inputs are copied in and chunk c-1's outputs copied back, on
- * two copy streams the library keeps per device (created on first use,
- * destroyed by vidattn_release), while chunk c's forward runs on `stream`;
- * events order the three steps of each chunk, and `stream` waits for the
- * last copy.  Either way the host outputs are valid once `stream` has been
+ * two copy streams the library keeps per device, while chunk c's forward
+ * runs, alternately on `stream` and on a third library stream (all created
+ * on first use, destroyed by vidattn_release); events order the three steps
+ * of each chunk, and `stream` waits for the last copy.  Either way the host outputs are valid once `stream` has been
  * synchronised, and they equal vidattn_fwd's bit for bit.  Host buffers
  * should be pinned for the copies to overlap.  h_seg_q/h_seg_kv and
  * d_seg_q/d_seg_kv follow the NULL rule of vidattn_fwd.

@@ -172,7 +172,7 @@ def test_host_buffer_entry_point_matches_device_entry_point():
     c = runs_case(1, 2, ((300, 0), (50, 1), (10, 2)), 128, 43)
     out_d, lse_d = run_gpu(c)
     B, H, S, D = c["q"].shape
-    pin = lambda a: torch.from_numpy(a).pin_memory()
+    pin = lambda a: torch.from_numpy(a if a.flags.writeable else a.copy()).pin_memory()
     hq, hk, hv = (pin(c[n].view(np.int16)) for n in ("q", "k", "v"))
     hsq, hsk = pin(c["seg_q"]), pin(c["seg_kv"])
     hout = torch.empty((B, H, S, D), dtype=torch.int16).pin_memory()

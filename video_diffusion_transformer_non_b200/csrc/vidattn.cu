@@ -77,8 +77,9 @@ struct DeviceInfo {
   uint32_t attrs_set = 0;   // bit (kernel variant index) once its smem limit is raised
   int* err = nullptr;       // device address of g_device_error on this device
   int rope_grid[4] = {};    // persistent grid of each rope3d variant (SMs x resident CTAs)
-  // vidattn_fwd_host's copy streams (host-to-device, device-to-host)
-  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  // vidattn_fwd_host's copy streams (host-to-device, device-to-host) and
+  // its second compute stream
+  cudaStream_t copy_in = nullptr, copy_out = nullptr, compute2 = nullptr;
 };
 
 // Recently encoded tensor maps (per device): a call on the same buffers and
@@ -325,24 +326,21 @@ int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32
   return cudaGetLastError() == cudaSuccess ? VIDATTN_OK : VIDATTN_ERR_CUDA;
 }
 
-// The copy streams of vidattn_fwd_host on device dev (created on first use).
-bool copy_streams(int dev, cudaStream_t* in, cudaStream_t* out) {
+// The streams of vidattn_fwd_host on device dev (created on first use).
+bool host_streams(int dev, cudaStream_t* in, cudaStream_t* out, cudaStream_t* comp2) {
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceInfo& info = g_devices[dev];
-  if (!info.copy_in &&
-      cudaStreamCreateWithFlags(&info.copy_in, cudaStreamNonBlocking) != cudaSuccess)
-    return false;
-  if (!info.copy_out &&
-      cudaStreamCreateWithFlags(&info.copy_out, cudaStreamNonBlocking) != cudaSuccess)
-    return false;
+  for (cudaStream_t* sp : {&info.copy_in, &info.copy_out, &info.compute2})
+    if (!*sp && cudaStreamCreateWithFlags(sp, cudaStreamNonBlocking) != cudaSuccess) return false;
   *in = info.copy_in;
   *out = info.copy_out;
+  *comp2 = info.compute2;
   return true;
 }
 
 // Below this many bytes of copies, vidattn_fwd_host does not split the work.
 constexpr size_t kPipelineMinBytes = size_t(64) << 20;
-constexpr int kPipelineChunks = 4;
+constexpr int kPipelineChunks = 8;
 
 // One warp waits on an mbarrier that nothing ever arrives on, through the
 // attention kernel's bounded wait; it gives up after timeout_ns and reports.
@@ -564,14 +562,16 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
   }
 
   // Pipelined by chunks of heads: the copy-in of chunk c+1 and the copy-out
-  // of chunk c-1 run on two copy streams while chunk c's attention runs on
-  // `stream`; events order each chunk's copy-in, attention and copy-out.
-  // The heads are independent, so the result is the same, bit for bit.
+  // of chunk c-1 run on two copy streams while chunk c's attention runs;
+  // chunks alternate between `stream` and a second compute stream, so a
+  // chunk's CTAs take the SMs that the previous chunk's last wave leaves
+  // idle.  Events order each chunk's copy-in, attention and copy-out.  The
+  // heads are independent, so the result is the same, bit for bit.
   int dev = 0;
   st = ensure_device(&dev);
   if (st != VIDATTN_OK) return st;
-  cudaStream_t cin = nullptr, cout = nullptr;
-  if (!copy_streams(dev, &cin, &cout)) return VIDATTN_ERR_CUDA;
+  cudaStream_t cin = nullptr, cout = nullptr, comp2 = nullptr;
+  if (!host_streams(dev, &cin, &cout, &comp2)) return VIDATTN_ERR_CUDA;
   const int hc = (H + kPipelineChunks - 1) / kPipelineChunks;
   const size_t hq = size_t(S_q) * D * 2, hkv = size_t(S_kv) * D * 2, hl = size_t(S_q) * 4;
   auto ev = [](cudaEvent_t* e) {
@@ -584,7 +584,9 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
   }
   bool ok = cudaEventRecord(start, stream) == cudaSuccess &&
             cudaStreamWaitEvent(cin, start, 0) == cudaSuccess &&
-            cudaStreamWaitEvent(cout, start, 0) == cudaSuccess;
+            cudaStreamWaitEvent(cout, start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(comp2, start, 0) == cudaSuccess;
+  int chunk = 0;
   auto* cq = static_cast<const char*>(h_q);
   auto* ck = static_cast<const char*>(h_k);
   auto* cv = static_cast<const char*>(h_v);
@@ -609,15 +611,16 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
                  cudaSuccess &&
              cudaMemcpyAsync(dv, cv + u * hkv, nh * hkv, cudaMemcpyHostToDevice, cin) ==
                  cudaSuccess)) &&
-           cudaEventRecord(in_done, cin) == cudaSuccess &&
-           cudaStreamWaitEvent(stream, in_done, 0) == cudaSuccess;
+           cudaEventRecord(in_done, cin) == cudaSuccess;
+      cudaStream_t comp = (chunk++ & 1) ? comp2 : stream;
+      ok = ok && cudaStreamWaitEvent(comp, in_done, 0) == cudaSuccess;
       if (ok) {
         st = vidattn_fwd(dq, dk, dv, d_seg_q ? d_seg_q + size_t(b) * S_q : nullptr,
                          d_seg_kv ? d_seg_kv + size_t(b) * S_kv : nullptr, dout, dl, 1, nh, S_q,
-                         S_kv, D, scale, stream_);
+                         S_kv, D, scale, reinterpret_cast<vidattn_stream_t>(comp));
         ok = st == VIDATTN_OK;
       }
-      ok = ok && cudaEventRecord(k_done, stream) == cudaSuccess &&
+      ok = ok && cudaEventRecord(k_done, comp) == cudaSuccess &&
            cudaStreamWaitEvent(cout, k_done, 0) == cudaSuccess &&
            cudaMemcpyAsync(static_cast<char*>(h_out) + u * hq, dout, nh * hq,
                            cudaMemcpyDeviceToHost, cout) == cudaSuccess &&
@@ -771,9 +774,9 @@ VIDATTN_API void vidattn_release(void) {
   cudaGetDevice(&prev);
   for (auto& kv : g_devices) {
     DeviceInfo& info = kv.second;
-    if (info.copy_in || info.copy_out) {
+    if (info.copy_in || info.copy_out || info.compute2) {
       cudaSetDevice(kv.first);
-      for (cudaStream_t* sp : {&info.copy_in, &info.copy_out}) {
+      for (cudaStream_t* sp : {&info.copy_in, &info.copy_out, &info.compute2}) {
         if (*sp) {
           cudaStreamSynchronize(*sp);
           cudaStreamDestroy(*sp);
