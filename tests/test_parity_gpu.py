@@ -299,7 +299,7 @@ def test_full_size_workload_sampled_rows(name):
     w = wl.WORKLOADS[name]
     c = wl.make_inputs(w)
     out, lse = run_gpu(c)
-    rows = sample_rows(w.B, w.H, w.S_q, w.segments, n_random=2048, n_heads_full=4)
+    rows = sample_rows(w.B, w.H, w.S_q, w.segments, n_random=4096, n_heads_full=8, seed=0)
     ro, rl = oracle.attn_rows(c["q"], c["k"], c["v"], rows, c["seg_q"], c["seg_kv"], c["scale"])
     b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
     idx = torch.from_numpy(((b * w.H + h) * w.S_q + i).astype(np.int64)).cuda()
