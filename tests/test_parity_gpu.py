@@ -143,6 +143,34 @@ def test_scale_zero_with_segments_gives_segment_means():
     check_all_rows(c, scale=0.0, what="scale 0 + ids")
 
 
+# ------------------------------------- more than 2048 key tiles with ids
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_ids_beyond_the_listed_tile_limit(causal):
+    """S_kv > 262144 (2048 key tiles) with ids: the roles walk the tile
+    summaries in global memory instead of a shared-memory list.  Queries
+    from every key segment plus an absent id; all rows against the oracle."""
+    B, H, D = 1, 2, 64
+    S_kv = 270000
+    seg_kv = np.concatenate([np.full(100000, 0), np.full(150000, 1),
+                             np.full(S_kv - 250000, 2)]).astype(np.int32)[None]
+    S_q = 600 if causal else 300
+    seg_q = np.array([0, 1, 2, 7])[np.arange(S_q) * 4 // S_q].astype(np.int32)[None]
+    c = wl.make_random(B, H, S_q, S_kv, D, 48, seg_q, seg_kv)
+    check_all_rows(c, what=f"beyond listed tiles causal={causal}", causal=causal)
+
+
+def test_ids_beyond_the_listed_tile_limit_two_samples():
+    B, H, D, S_q, S_kv = 2, 1, 128, 256, 263000
+    seg_kv = np.zeros((B, S_kv), np.int32)
+    seg_kv[0, 200000:] = 1
+    seg_kv[1, :1000] = 1
+    seg_q = np.zeros((B, S_q), np.int32)
+    seg_q[:, S_q // 2:] = 1
+    c = wl.make_random(B, H, S_q, S_kv, D, 49, seg_q, seg_kv)
+    check_all_rows(c, what="beyond listed tiles, B=2")
+
+
 # -------------------------------------------------------------- edge cases
 
 def test_empty_key_sequence():

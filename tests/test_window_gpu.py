@@ -69,6 +69,18 @@ def test_window_matches_oracle(name, clamped):
     check_window(c, win, f"{name} clamped={clamped}")
 
 
+def test_window_at_the_key_tile_limit():
+    """S_kv = 262144 keys (2048 key tiles, the most a window call takes): a
+    16 x 128 x 128 volume, window 3 x 3 x 5, queries of two frames."""
+    grid = (16, 128, 128)
+    ck = wl.raster_coords(grid, 1)
+    assert ck.shape[1] == 262144
+    cq = np.ascontiguousarray(ck[:, 7 * 16384: 7 * 16384 + 512])   # frame 7, first 4 rows
+    c = wl.make_random(1, 1, cq.shape[1], ck.shape[1], 64, 30)
+    win = dict(coord_q=cq, coord_kv=ck, size=(3, 3, 5), extent=grid, clamped=True)
+    check_window(c, win, "2048 key tiles")
+
+
 def test_unit_window_returns_own_value():
     c, win = volume_case(1, 2, 128, (3, 10, 20), (1, 1, 1), False, seed=21)
     out, lse = run_window(c, win)
