@@ -191,3 +191,25 @@ def test_full_480p_q_k_sampled_tokens(interleaved):
         xs = np.ascontiguousarray(x[:, :, rows])
         ref = rope3d_f64(xs, grid, bands, interleaved=interleaved, S=w.S, rows=rows)
         check(got, xs, ref, f"480p {what}")
+
+
+@pytest.mark.parametrize("interleaved", [True, False])
+def test_rope_then_attention_matches_oracle(interleaved):
+    """The benchmark's --rope step on a small case: q and k rotated on the
+    GPU, then attention on the rotated tensors, against the oracle's
+    attention on the oracle's rotation rounded to bf16 (the rotation's output
+    precision), under the attention tolerances."""
+    import oracle
+    from _gpu_helpers import bf16_to_f64, compare
+    grid, bands = (2, 6, 9), (44, 42, 42)
+    S = 108 + 20                                  # video tokens, then 20 text tokens
+    c = wl.make_random(1, 2, S, S, 128, 50)
+    q, k, v = to_dev_bf16(c["q"]), to_dev_bf16(c["k"]), to_dev_bf16(c["v"])
+    qr, kr = binding.rope3d(q, k, grid, bands, interleaved=interleaved)
+    out, lse = binding.attention(qr, kr, v, scale=c["scale"])
+    torch.cuda.synchronize()
+    to_bits = lambda x: wl.f32_to_bf16_bits(x.astype(np.float32))
+    rq = to_bits(rope3d_f64(c["q"], grid, bands, interleaved=interleaved))
+    rk = to_bits(rope3d_f64(c["k"], grid, bands, interleaved=interleaved))
+    ro, rl = oracle.attn_fwd(rq, rk, c["v"], scale=c["scale"])
+    compare(bf16_to_f64(out), lse.double().cpu().numpy(), ro, rl, "rope then attention")
