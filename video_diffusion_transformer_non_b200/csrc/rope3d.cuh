@@ -13,8 +13,9 @@
 // (the angles in fp64, reduced to [-pi, pi], then sincosf; two tables
 // alternate, so one barrier per tile suffices), each thread keeps the entries
 // of its own 8 features in registers and then streams 16-byte chunks of all
-// slabs through them: kRopeUnroll loads in flight per thread, streaming-cache
-// loads and stores (every byte is touched once).  The
+// slabs through them: 8 loads in flight per thread (4 with the half-split
+// pairing, whose staging needs more registers), streaming-cache loads and
+// stores (every byte is touched once).  The
 // interleaved pairing finds both features of a pair in one chunk; the
 // half-split pairing stages the chunk in shared memory and reads the partner
 // feature from the neighbouring thread of the same row.
@@ -29,7 +30,6 @@ namespace vidattn {
 
 constexpr int kRopeThreads = 256;
 constexpr int kRopeTokens = 8;
-constexpr int kRopeUnroll = 4;
 constexpr int kRopeMaxD = 128;
 
 // n / d for 0 <= n < 2^31 by one multiply-high, add and shift (Granlund and
@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope3d_kernel(const __grid_const
   constexpr int kPerSlab = kRopeTokens * kChunks;          // threads per slab
   constexpr int kSlabsPerPass = kRopeThreads / kPerSlab;
   static_assert(kRopeThreads % kPerSlab == 0 && 32 % kChunks == 0, "tile shape");
+  constexpr int kRopeUnroll = kInterleaved ? 8 : 4;   // 16-byte loads in flight per thread
 
   __shared__ __align__(16) float2 table[2][kRopeTokens][kHalf];
   __shared__ uint4 stage[kInterleaved ? 1 : kRopeUnroll][kRopeThreads];
