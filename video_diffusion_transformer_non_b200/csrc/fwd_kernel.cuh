@@ -1,36 +1,46 @@
-// Segment-masked, non-causal attention forward for sm_100a.
+// Masked multi-head attention forward for sm_100a.
 //
-// Computes, per (b, h, query row i), softmax over the keys j whose segment id
-// equals the query's (all keys when no ids are given) of scale * q_i . k_j,
-// applied to v, plus the natural log-sum-exp of the allowed scaled logits.
-// The full query-key matrix is never stored: scores live only in tensor memory
-// one 128x128 tile at a time and an online softmax carries the running max and
-// sum (vidax: A Unified JAX Framework for Video Generative Models on
-// Accelerator Meshes, §2 "3D RoPE, 3D VAEs, and flash attention", which
-// dispatches such attention to flash-attention kernels, its reference [2]);
-// key tiles whose ids cannot match any query of the CTA are skipped, not
-// masked (same paper, Appendix A, Table 4, group 2, row "HunyuanVideo-1.5:
-// RESOURCE_EXHAUSTED at 720p").
+// Computes, per (b, h, query row i), softmax over the keys j visible to the
+// query of scale * q_i . k_j, applied to v, plus the natural log-sum-exp of
+// the visible scaled logits.  A key is visible when the segment ids match
+// (every key when no ids are given), and, with the options, when it lies
+// within the causal limit j <= i + (S_kv - S_q) or in the query's 3D
+// neighbourhood window.  The full query-key matrix is never stored: scores
+// live only in tensor memory one 128x128 tile at a time and an online softmax
+// carries the running offset and sum (vidax: A Unified JAX Framework for
+// Video Generative Models on Accelerator Meshes, §2 "3D RoPE, 3D VAEs, and
+// flash attention", which dispatches such attention to flash-attention
+// kernels, its reference [2]); key tiles that no query of the CTA can see are
+// skipped, not masked (same paper, Appendix A, Table 4, group 2, row
+// "HunyuanVideo-1.5: RESOURCE_EXHAUSTED at 720p").
 //
 // One CTA = (b, h, 256 query rows as two 128-row tiles Q0, Q1).  384 threads:
 //   warps 0-3  softmax for Q0 (TMEM lanes 0-127 = the tile's rows)
 //   warps 4-7  softmax for Q1
-//   warp  8    allocates TMEM; lane 0 issues every tcgen05.mma and commit
-//   warp  9    lane 0 issues every TMA load (Q0, Q1 once; then K_j, V_j)
+//   warp  8    allocates TMEM; runs the tensor-core schedule converged, an
+//              elected lane issuing every tcgen05.mma and commit
+//   warp  9    runs the load schedule converged, an elected lane issuing
+//              every TMA load (Q0, Q1 once; then K_j, V_j)
 //   warps 10-11 idle
-// Tensor memory (512 columns x 128 lanes, fp32):
-//   [0,128) S0 / P0   [128,256) S1 / P1   [256,256+D) O0   [256+D,256+2D) O1
+// Tensor memory (512 columns x 128 lanes, fp32), D = 128:
+//   [0,128) S0 / P0   [128,256) S1 / P1   [256,384) O0   [384,512) O1
 // P (bf16, two per column) overwrites the first 64 columns of its S tile.
+// D = 64 (kSepP): S0, S1 in [0,256), P0, P1 in [256,384), O0, O1 in [384,512);
+// the softmax moves its S row into registers and releases S at once.
 // Shared memory: Q0, Q1, then a ring of kStages K-or-V tiles; every tile is
 // [D/64][128 rows][64 columns] bf16 written by TMA with 128-byte swizzle.
 //
-// Tensor-core order (one thread, in issue order; each tile pair t):
+// Tensor-core order for D = 128 (in issue order; each tile pair t):
 //   S0 = Q0 K_0^T, S1 = Q1 K_0^T, then for t = 0..n-1:
 //   O0 += P0 V_t, S0 = Q0 K_{t+1}^T, O1 += P1 V_t, S1 = Q1 K_{t+1}^T
 // so the tensor core works on one Q tile while the other's softmax runs.
-// The running max is updated lazily: O is rescaled only when a row's max
-// grows by more than 2^8 (the exponentials stay <= 256 otherwise), which
-// makes the O read-modify-write in tensor memory rare.
+// The softmax uses a running offset: after a row's first tile P = 2^(c s - m)
+// with the row's previous offset m and no tile maximum; only a tile whose sum
+// of P exceeds 2^32, a masked tile (except in the kMaskFast variant), a row's
+// first tile or scale <= 0 takes the exact path (tile maximum; O and the row
+// sum rescaled when the maximum grows by more than 2^8).  A masked tile's key
+// ids or coordinates are staged per warp in shared memory and each row builds
+// a 128-bit mask from them.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
