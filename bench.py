@@ -23,6 +23,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -54,11 +55,18 @@ KERNEL_SOURCES = ["fwd_kernel.cuh", "ptx.cuh", "classify.cuh"]
 ROPE_SOURCES = ["rope3d.cuh", "ptx.cuh"]
 
 
+def code_only(src: str) -> str:
+    """C++ source without comments and blank lines: what the compiler sees."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def measured_traffic(w, summary=None, sources=KERNEL_SOURCES):
     """DRAM bytes per launch from the committed ncu summary of this workload's
-    kernel, or None when there is none or the kernel sources changed since."""
+    kernel, or None when there is none or the kernel's code changed since
+    (sha256 over its device sources with comments removed)."""
     import hashlib
-    import re
     path = os.path.join(ROOT, "profiles",
                         summary or f"vidattn_fwd_kernel_d{w.D}__{w.name}_h8.md")
     if not os.path.exists(path):
@@ -71,8 +79,8 @@ def measured_traffic(w, summary=None, sources=KERNEL_SOURCES):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "video_diffusion_transformer_non_b200", "csrc")
     for f in sources:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f)) as fh:
+            h.update(code_only(fh.read()).encode())
     return int(val.group(1)) if h.hexdigest() == sha.group(1) else None
 
 
