@@ -1,6 +1,11 @@
 /*
- * vidattn: segment-masked, non-causal multi-head attention forward for video
- * diffusion transformers, on NVIDIA B200 (sm_100a).
+ * vidattn: the multi-head attention forward of video diffusion transformers,
+ * on NVIDIA B200 (sm_100a) — bidirectional attention masked by segment ids
+ * (vidattn_fwd), with an optional causal limit (vidattn_fwd_ex) or a 3D
+ * neighbourhood window (vidattn_fwd_window) — and the 3D rotary embedding of
+ * q and k ahead of it (vidattn_rope3d).
+ *
+ * The base operation:
  *
  * The operation (vidax: A Unified JAX Framework for Video Generative Models on
  * Accelerator Meshes, §2 "3D RoPE, 3D VAEs, and flash attention": full

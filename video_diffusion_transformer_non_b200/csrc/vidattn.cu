@@ -1,6 +1,8 @@
 // Host side of the vidattn C ABI: argument checks, TMA descriptors, the
-// segment-summary scratch cache, and kernel launches.  The operation and the
-// argument contract are documented in include/vidattn.h.
+// tile-summary scratch cache, kernel launches (attention, causal and window
+// variants, tile summaries, the rotary embedding), and the host-buffer entry
+// point's copy pipeline.  The operations and the argument contracts are
+// documented in include/vidattn.h.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
