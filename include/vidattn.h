@@ -5,9 +5,7 @@
  * neighbourhood window (vidattn_fwd_window) — and the 3D rotary embedding of
  * q and k ahead of it (vidattn_rope3d).
  *
- * The base operation:
- *
- * The operation (vidax: A Unified JAX Framework for Video Generative Models on
+ * The base operation (vidax: A Unified JAX Framework for Video Generative Models on
  * Accelerator Meshes, §2 "3D RoPE, 3D VAEs, and flash attention": full
  * self-attention over multi-frame patch volumes, computed without storing the
  * query-key matrix, after FlashAttention, its reference [2]; Appendix A,
