@@ -87,17 +87,21 @@ def test_unit_window_returns_own_value():
     assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), c["v"])
 
 
-def test_covering_window_equals_plain_attention_bitwise():
+def test_covering_window_equals_plain_attention():
     """A window wider than the volume is full attention: on a volume of whole
-    key tiles (512 tokens) no tile is masked, so the bits equal vidattn_fwd's."""
+    key tiles (512 tokens) no tile is masked, so the result is vidattn_fwd's
+    up to the rounding of the exponentials (the window kernel computes 2 of
+    16 on the FMA pipe, the plain kernel 4), and the oracle's."""
     grid = (4, 8, 16)
     c, win = volume_case(1, 2, 128, grid, (7, 15, 31), False, seed=22)
     out, lse = run_window(c, win)
     plain_o, plain_l = binding.attention(to_dev_bf16(c["q"]), to_dev_bf16(c["k"]),
                                          to_dev_bf16(c["v"]), scale=c["scale"])
     torch.cuda.synchronize()
-    assert torch.equal(out.view(torch.int16), plain_o.view(torch.int16))
-    assert torch.equal(lse, plain_l)
+    d = (out.float() - plain_o.float()).abs()
+    assert float(d.max()) <= 8e-3 and float(d.mean()) <= 5e-4
+    assert float((lse - plain_l).abs().max()) <= 2e-4
+    check_window(c, win, "covering, whole tiles")
 
 
 def test_covering_window_on_a_ragged_volume():

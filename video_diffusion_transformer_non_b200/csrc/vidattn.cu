@@ -123,9 +123,11 @@ FwdKernel fwd_variant(int e) {
   }
 }
 // 3D neighbourhood windows: masked tiles on the running-offset path (D = 128,
-// the default 4 of 16 exponentials on the FMA pipe); D = 64 uses the default.
+// 2 of 16 exponentials on the FMA pipe: the mask work takes issue slots, and
+// 2 measured 3 % faster than 4 on the 11^3 window over the 480p volume);
+// D = 64 uses the default kernel.
 FwdKernel fwd_window_variant(int D) {
-  return D == 128 ? vidattn_fwd_kernel<128, 4, true> : vidattn_fwd_kernel<64, 2, false>;
+  return D == 128 ? vidattn_fwd_kernel<128, 2, true> : vidattn_fwd_kernel<64, 2, false>;
 }
 // Default share of exponentials moved off the MUFU unit (measured best on
 // B200: 4 of 16 at D = 128, 2 of 16 at D = 64, where the FMA-pipe version's
