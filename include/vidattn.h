@@ -307,9 +307,10 @@ VIDATTN_API int vidattn_kernels_per_call(const int32_t* seg_q, const int32_t* se
  * hangs; the CUDA context stays usable. */
 VIDATTN_API int vidattn_selftest_timeout(int timeout_us, vidattn_stream_t stream);
 
-/* Frees the library's scratch buffers on every device after synchronising
- * the streams they belong to.  Safe to call at any time; later calls
- * allocate again on demand. */
+/* Frees the library's scratch buffers and destroys its internal streams (the
+ * copy and second compute streams of vidattn_fwd_host) on every device, after
+ * synchronising the streams concerned.  Call it while no other thread is
+ * inside a vidattn call; later calls allocate again on demand. */
 VIDATTN_API void vidattn_release(void);
 
 /* Library version and the GPU architecture it was compiled for. */
