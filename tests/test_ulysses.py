@@ -114,3 +114,120 @@ def test_ulysses_single_gpu_world_equals_kernel():
         assert torch.equal(l1, l2)
     finally:
         dist.destroy_process_group()
+
+
+def _oracle_attn_win(q, k, v, seg_q, seg_kv, scale, causal, window=None):
+    """Per-shard window attention on the CPU: the fp64 oracle's window rule."""
+    import oracle
+    to_bits = lambda t: t.numpy().view(np.uint16)
+    c = window["coords"].numpy()
+    win = dict(coord_q=c, coord_kv=c.copy(), size=window["size"], extent=window["extent"],
+               clamped=window["clamped"])
+    out, lse = oracle.attn_fwd(to_bits(q), to_bits(k), to_bits(v), None, None, scale,
+                               window=win)
+    return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+def _oracle_rope(q, k, rope):
+    """Per-shard rotation on the CPU: the fp64 oracle, rounded to bf16 as the
+    kernel stores it (bit patterns carried in float16-typed tensors)."""
+    from oracle.rope3d import rope3d_f64
+    from video_diffusion_transformer_non_b200 import workloads as wl
+    out = []
+    for t in (q, k):
+        r = rope3d_f64(t.numpy().view(np.uint16), rope["grid"], rope["bands"],
+                       rope.get("theta", 10000.0), rope.get("interleaved", True),
+                       rope.get("offset", 0))
+        out.append(torch.from_numpy(wl.f32_to_bf16_bits(r.astype(np.float32)).view(np.float16)))
+    return out[0], out[1]
+
+
+def _rank_main_win(rank, world, port, case, coords, window, rope, n_chunks, q_out):
+    import torch.distributed as dist
+    from video_diffusion_transformer_non_b200.ulysses import ulysses_attention
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        S = case["q"].shape[2]
+        Sl = S // world
+        sl = slice(rank * Sl, (rank + 1) * Sl)
+        shard = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, :, sl]).view(np.float16))
+        win = dict(window, coords=torch.from_numpy(np.ascontiguousarray(coords[:, sl])))
+        out, lse = ulysses_attention(shard(case["q"]), shard(case["k"]), shard(case["v"]), None,
+                                     case["scale"], False, None, n_chunks, _oracle_attn_win,
+                                     window=win, rope=rope, rope_fn=_oracle_rope)
+        q_out.put((rank, out.numpy(), lse.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,n_chunks,clamped", [(2, 1, True), (4, 2, False)])
+def test_ulysses_window_with_rope_matches_whole_sequence(world, n_chunks, clamped):
+    """3D neighbourhood attention of rotated q and k under sequence
+    parallelism equals the whole-sequence computation (rotation at global
+    positions, windows over all tokens)."""
+    import oracle
+    from oracle.rope3d import rope3d_f64
+    from video_diffusion_transformer_non_b200 import workloads as wl
+    grid, bands = (2, 4, 6), (4, 6, 6)
+    B, H, D = 1, 8, 16
+    S = int(np.prod(grid))
+    case = wl.make_random(B, H, S, S, D, 62)
+    coords = wl.raster_coords(grid, B)
+    window = dict(size=(3, 3, 3), extent=grid, clamped=clamped)
+    rope = dict(grid=grid, bands=bands, theta=10000.0, interleaved=True, offset=0)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_win,
+                         args=(r, world, port, case, coords, window, rope, n_chunks, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=60) for _ in range(world)], key=lambda x: x[0])
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    out = np.concatenate([r[1] for r in res], axis=2)
+    lse = np.concatenate([r[2] for r in res], axis=2)
+    rot = lambda x: wl.f32_to_bf16_bits(rope3d_f64(x, grid, bands).astype(np.float32))
+    win = dict(coord_q=coords, coord_kv=coords.copy(), size=window["size"], extent=grid,
+               clamped=clamped)
+    ro, rl = oracle.attn_fwd(rot(case["q"]), rot(case["k"]), case["v"], scale=case["scale"],
+                             window=win)
+    assert np.max(np.abs(out - ro)) <= 1e-12
+    assert np.max(np.abs(lse - rl)) <= 1e-12
+
+
+@pytest.mark.gpu
+def test_ulysses_single_gpu_window_with_rope_equals_direct_calls():
+    """World of one over NCCL, window + rotary embedding: bitwise the RoPE
+    pass followed by the window kernel."""
+    import torch.distributed as dist
+    from video_diffusion_transformer_non_b200 import binding
+    from video_diffusion_transformer_non_b200 import workloads as wl
+    from video_diffusion_transformer_non_b200.ulysses import ulysses_attention
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        grid, bands = (3, 8, 20), (44, 42, 42)
+        B, H, D = 1, 4, 128
+        S = int(np.prod(grid))
+        c = wl.make_random(B, H, S, S, D, 63)
+        up = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+        q, k, v = up(c["q"]), up(c["k"]), up(c["v"])
+        co = torch.from_numpy(wl.raster_coords(grid, B).copy()).cuda()
+        window = dict(coords=co, size=(3, 5, 5), extent=grid, clamped=True)
+        rope = dict(grid=grid, bands=bands)
+        q0, k0 = q.clone(), k.clone()
+        o1, l1 = ulysses_attention(q, k, v, None, c["scale"], n_chunks=2, window=window,
+                                   rope=rope)
+        torch.cuda.synchronize()
+        assert torch.equal(q, q0) and torch.equal(k, k0)     # the inputs are left as they were
+        qr, kr = binding.rope3d(q, k, grid, bands)
+        o2, l2 = binding.attention_window(qr, kr, v, co, co, (3, 5, 5), grid, True, c["scale"])
+        torch.cuda.synchronize()
+        assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+        assert torch.equal(l1, l2)
+    finally:
+        dist.destroy_process_group()

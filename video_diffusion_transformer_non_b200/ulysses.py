@@ -19,6 +19,12 @@ exchange of one chunk overlaps the attention of the previous one (NCCL runs
 the collectives on its own stream).  The collective is torch.distributed's
 (NCCL over NVLink on GPUs, gloo on CPU for the tests); the data-path kernel is
 vidattn's.  `attn_fn` replaces the attention call (tests on CPU).
+
+The other attention forms go through the same exchange: a 3D neighbourhood
+window (each rank's token coordinates are all-gathered like the ids) and the
+3D rotary embedding, which is applied after the exchange, where each rank
+holds the whole sequence of its heads, so positions are the global ones;
+`rope_fn` replaces the rotation (tests on CPU).
 """
 from __future__ import annotations
 
@@ -70,35 +76,59 @@ def _heads_to_seq(y: torch.Tensor, P: int, group) -> _Exchange:
                      .contiguous(), P, group)
 
 
-def _cuda_attention(q, k, v, seg_q, seg_kv, scale, causal):
+def _cuda_attention(q, k, v, seg_q, seg_kv, scale, causal, window=None):
+    if window is not None:
+        return binding.attention_window(q, k, v, window["coords"], window["coords"],
+                                        window["size"], window["extent"], window["clamped"],
+                                        scale)
     return binding.attention(q, k, v, seg_q, seg_kv, scale, causal=causal)
 
 
+def _cuda_rope(q, k, rope):
+    # out of place: without an exchange (one rank) q and k are views of the
+    # caller's tensors, which must not change
+    return binding.rope3d(q, k, rope["grid"], rope["bands"], theta=rope.get("theta", 10000.0),
+                          interleaved=rope.get("interleaved", True),
+                          token_offset=rope.get("offset", 0))
+
+
+def _all_gather_seq(x, P, group):
+    """[B, S/P] per rank -> [B, S] in rank order."""
+    if P == 1:
+        return x.contiguous()
+    parts = [torch.empty_like(x) for _ in range(P)]
+    dist.all_gather(parts, x.contiguous(), group=group)
+    return torch.cat(parts, dim=1).contiguous()
+
+
 def ulysses_attention(q, k, v, seg=None, scale=None, causal=False, group=None, n_chunks=1,
-                      attn_fn=None):
+                      attn_fn=None, window=None, rope=None, rope_fn=None):
     """Attention over a sequence sharded across the ranks of `group`.
 
     q, k, v: [B, H, S/P, D] (this rank's contiguous sequence shard; H divisible
-    by P * n_chunks); seg: int32 [B, S/P] or None.  Returns (out [B, H, S/P, D],
-    lse fp32 [B, H, S/P]) for this rank's shard, equal to the corresponding
-    rows of single-device attention over the whole sequence.  Head chunk c's
-    attention starts once its own inputs have arrived, while later chunks'
-    exchanges are still in flight."""
+    by P * n_chunks); seg: int32 [B, S/P] or None.  window: dict(coords=int32
+    [B, S/P] packed t << 22 | h << 11 | w of this rank's tokens, size, extent,
+    clamped) for 3D neighbourhood attention, or None.  rope: dict(grid, bands,
+    theta, interleaved, offset) to rotate q and k (global positions) before
+    the attention, or None.  Returns (out [B, H, S/P, D], lse fp32 [B, H, S/P])
+    for this rank's shard, equal to the corresponding rows of single-device
+    attention over the whole sequence.  Head chunk c's attention starts once
+    its own inputs have arrived, while later chunks' exchanges are still in
+    flight."""
     P = _world(group)
     B, H, Sl, D = q.shape
     if H % (P * n_chunks):
         raise ValueError(f"H={H} must be divisible by world size {P} x chunks {n_chunks}")
     if scale is None:
         scale = D ** -0.5
+    if window is not None and (seg is not None or causal):
+        raise ValueError("a window goes without ids and without the causal limit")
     attn = attn_fn or _cuda_attention
-    seg_full = None
-    if seg is not None:
-        if P == 1:
-            seg_full = seg.contiguous()
-        else:
-            parts = [torch.empty_like(seg) for _ in range(P)]
-            dist.all_gather(parts, seg.contiguous(), group=group)
-            seg_full = torch.cat(parts, dim=1).contiguous()
+    turn = rope_fn or _cuda_rope
+    seg_full = None if seg is None else _all_gather_seq(seg, P, group)
+    win_full = None
+    if window is not None:
+        win_full = dict(window, coords=_all_gather_seq(window["coords"], P, group))
     Hc = H // n_chunks
     inputs = []
     for c in range(n_chunks):          # every input exchange goes out first
@@ -107,7 +137,12 @@ def ulysses_attention(q, k, v, seg=None, scale=None, causal=False, group=None, n
     outputs = []
     for c in range(n_chunks):
         qh, kh, vh = (x.result() for x in inputs[c])
-        o, l = attn(qh, kh, vh, seg_full, seg_full, scale, causal)
+        if rope is not None:
+            qh, kh = turn(qh, kh, rope)
+        if win_full is not None:
+            o, l = attn(qh, kh, vh, None, None, scale, False, window=win_full)
+        else:
+            o, l = attn(qh, kh, vh, seg_full, seg_full, scale, causal)
         outputs.append((_heads_to_seq(o, P, group), _heads_to_seq(l, P, group)))
     outs = [o.result() for o, _ in outputs]
     lses = [l.result() for _, l in outputs]
