@@ -189,3 +189,101 @@ def test_window_argument_errors_return_before_any_launch(lib, kw, expect):
 
 def test_window_empty_query_is_a_no_op(lib):
     assert win(lib, Sq=0) == OK
+
+
+# --- the Python helpers' tensor checks ---------------------------------------
+# The helpers (attention, attention_window, rope3d) check dtype, device,
+# layout and shapes before a pointer reaches the library.  Here the device
+# type the checks require is "cpu", and the library is replaced by one that
+# fails the test when touched, so every case below must raise first.
+
+@pytest.fixture
+def host_checks(monkeypatch):
+    torch = pytest.importorskip("torch")
+
+    def no_library():
+        raise AssertionError("an invalid call reached the library")
+    monkeypatch.setattr(binding, "_DEVICE_TYPE", "cpu")
+    monkeypatch.setattr(binding, "load_library", no_library)
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)
+    return torch, bf, i32
+
+
+def test_helpers_refuse_host_tensors_where_a_device_is_required():
+    torch = pytest.importorskip("torch")
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.attention(q, q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.rope3d(q, q, (1, 2, 4), (22, 22, 20))
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.attention_window(q, q, q, torch.zeros(1, 8, dtype=torch.int32),
+                                 torch.zeros(1, 8, dtype=torch.int32), (3, 3, 3), (1, 2, 4))
+
+
+@pytest.mark.parametrize("case", [
+    "dtype", "ndim", "strided", "kv_shape", "d_mismatch", "seg_one", "seg_dtype", "seg_shape",
+    "not_tensor"])
+def test_attention_helper_checks(host_checks, case):
+    torch, bf, i32 = host_checks
+    q, k, v = bf(1, 2, 8, 64), bf(1, 2, 16, 64), bf(1, 2, 16, 64)
+    sq, sk = i32(1, 8), i32(1, 16)
+    if case == "dtype":
+        q = q.float()
+    elif case == "ndim":
+        q = q[0]
+    elif case == "strided":
+        q = bf(1, 8, 2, 64).transpose(1, 2)
+    elif case == "kv_shape":
+        v = bf(1, 2, 15, 64)
+    elif case == "d_mismatch":
+        k, v = bf(1, 2, 16, 128), bf(1, 2, 16, 128)
+    elif case == "seg_one":
+        sk = None
+    elif case == "seg_dtype":
+        sq = sq.long()
+    elif case == "seg_shape":
+        sk = i32(1, 8)
+    elif case == "not_tensor":
+        k = [0]
+    with pytest.raises(ValueError):
+        binding.attention(q, k, v, sq, sk)
+
+
+@pytest.mark.parametrize("case", ["no_coords", "coord_dtype", "coord_shape"])
+def test_window_helper_checks(host_checks, case):
+    torch, bf, i32 = host_checks
+    q = bf(1, 2, 8, 64)
+    cq, ck = i32(1, 8), i32(1, 8)
+    if case == "no_coords":
+        cq = ck = None
+    elif case == "coord_dtype":
+        ck = ck.long()
+    elif case == "coord_shape":
+        cq = i32(2, 8)
+    with pytest.raises(ValueError):
+        binding.attention_window(q, q, q, cq, ck, (3, 3, 3), (1, 2, 4))
+
+
+@pytest.mark.parametrize("case", ["dtype", "k_shape", "k_strides", "feature_stride", "out_shape",
+                                  "out_k_alone"])
+def test_rope_helper_checks(host_checks, case):
+    torch, bf, i32 = host_checks
+    q, k = bf(1, 2, 8, 64), bf(1, 2, 8, 64)
+    kw = {}
+    if case == "dtype":
+        k = k.half()
+    elif case == "k_shape":
+        k = bf(1, 2, 9, 64)
+    elif case == "k_strides":
+        k = bf(1, 8, 2, 64).transpose(1, 2)
+    elif case == "feature_stride":
+        q = k = bf(1, 2, 64, 8).transpose(2, 3)
+    elif case == "out_shape":
+        kw["out_q"] = bf(1, 2, 8, 128)
+    elif case == "out_k_alone":
+        k = None
+        kw["out_k"] = bf(1, 2, 8, 64)
+    with pytest.raises(ValueError):
+        binding.rope3d(q, k, (1, 2, 4), (22, 22, 20), **kw)

@@ -17,6 +17,8 @@ _HEADER = os.path.join(os.path.dirname(_PKG), "include", "vidattn.h")
 
 VIDATTN_OK = 0
 _lib = None
+# the device type the tensor helpers require (the library reads device memory)
+_DEVICE_TYPE = "cuda"
 
 
 def library_path() -> str:
@@ -101,6 +103,57 @@ def _stream(stream):
     return stream.cuda_stream
 
 
+def _check_tensors(named, dtype, ndim=None, contiguous=True):
+    """Raise ValueError unless every tensor in ``named`` (name -> tensor or
+    None) is a CUDA tensor of ``dtype`` on one device, ``ndim``-dimensional
+    and (when asked) contiguous.  Runs before any pointer reaches the library,
+    whose kernels read device memory in the documented layout only."""
+    import torch
+    device = None
+    for name, t in named.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise ValueError(f"{name} must be a torch tensor, not {type(t).__name__}")
+        if t.device.type != _DEVICE_TYPE:
+            raise ValueError(f"{name} must be on a CUDA device (is on {t.device})")
+        if device is None:
+            device = t.device
+        elif t.device != device:
+            raise ValueError(f"{name} is on {t.device}, the other tensors on {device}")
+        if t.dtype != dtype:
+            raise ValueError(f"{name} must be {dtype} (is {t.dtype})")
+        if ndim is not None and t.dim() != ndim:
+            raise ValueError(f"{name} must have {ndim} dims (has shape {tuple(t.shape)})")
+        if contiguous and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def _check_qkv(q, k, v):
+    """q bf16 [B,H,S_q,D], k and v bf16 [B,H,S_kv,D], contiguous, on one GPU."""
+    import torch
+    _check_tensors(dict(q=q, k=k, v=v), torch.bfloat16, ndim=4)
+    if k.shape != v.shape or k.shape[:2] != q.shape[:2] or k.shape[3] != q.shape[3]:
+        raise ValueError(f"shapes do not match: q {tuple(q.shape)}, k {tuple(k.shape)}, "
+                         f"v {tuple(v.shape)}")
+
+
+def _check_per_token(name_q, t_q, name_kv, t_kv, B, S_q, S_kv, device):
+    """int32 [B,S_q] and [B,S_kv] per-token arrays (ids or coordinates), both
+    or neither, contiguous, on the device of q."""
+    import torch
+    if (t_q is None) != (t_kv is None):
+        raise ValueError(f"{name_q} and {name_kv} must both be given or both be None")
+    if t_q is None:
+        return
+    _check_tensors({name_q: t_q, name_kv: t_kv}, torch.int32, ndim=2)
+    if t_q.device != device:
+        raise ValueError(f"{name_q} is on {t_q.device}, q on {device}")
+    if tuple(t_q.shape) != (B, S_q) or tuple(t_kv.shape) != (B, S_kv):
+        raise ValueError(f"{name_q} must be [B,S_q] = {(B, S_q)} and {name_kv} [B,S_kv] = "
+                         f"{(B, S_kv)} (are {tuple(t_q.shape)}, {tuple(t_kv.shape)})")
+
+
 def vidattn_fwd(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D, scale, stream=None) -> int:
     """Enqueue the forward on ``stream`` (device pointers).  Returns the status."""
     return load_library().vidattn_fwd(
@@ -158,8 +211,10 @@ def attention(q, k, v, seg_q=None, seg_kv=None, scale=None, stream=None, causal=
     q: bf16 [B,H,S_q,D]; k, v: bf16 [B,H,S_kv,D]; seg_*: int32 [B,S] or None.
     Returns (out bf16 [B,H,S_q,D], lse fp32 [B,H,S_q]); raises on error."""
     import torch
+    _check_qkv(q, k, v)
     B, H, S_q, D = q.shape
     S_kv = k.shape[2]
+    _check_per_token("seg_q", seg_q, "seg_kv", seg_kv, B, S_q, S_kv, q.device)
     if scale is None:
         scale = D ** -0.5
     out = torch.empty_like(q)
@@ -191,6 +246,10 @@ def rope3d(q, k=None, grid=None, bands=None, theta=10000.0, interleaved=True, to
     works); grid = (T, Hg, Wg) of the video tokens; bands = (d_t, d_h, d_w).
     ``out_q=q`` (and ``out_k=k``) rotates a contiguous input in place."""
     import torch
+    _check_tensors(dict(q=q, k=k, out_q=out_q, out_k=out_k), torch.bfloat16, ndim=4,
+                   contiguous=False)
+    if out_k is not None and k is None:
+        raise ValueError("out_k without k")
     B, H, S, D = q.shape
     if k is not None and k.shape != q.shape:
         raise ValueError("q and k must have the same shape")
@@ -232,8 +291,12 @@ def attention_window(q, k, v, coord_q, coord_kv, size, extent, clamped=True, sca
     """3D neighbourhood attention.  coord_*: int32 [B,S] packed t << 22 | h << 11 | w;
     size = (win_t, win_h, win_w), odd; extent = (T, Hg, Wg).  Returns (out, lse)."""
     import torch
+    _check_qkv(q, k, v)
     B, H, S_q, D = q.shape
     S_kv = k.shape[2]
+    if coord_q is None or coord_kv is None:
+        raise ValueError("a window needs coord_q and coord_kv")
+    _check_per_token("coord_q", coord_q, "coord_kv", coord_kv, B, S_q, S_kv, q.device)
     if scale is None:
         scale = D ** -0.5
     out = torch.empty_like(q)
