@@ -184,8 +184,10 @@ VIDATTN_API int vidattn_fwd_window(const void* q, const void* k, const void* v,
  * two copy streams the library keeps per device, while chunk c's forward
  * runs, alternately on `stream` and on a third library stream (all created
  * on first use, destroyed by vidattn_release); events order the three steps
- * of each chunk, and `stream` waits for the last copy.  Either way the host outputs are valid once `stream` has been
- * synchronised, and they equal vidattn_fwd's bit for bit.  Host buffers
+ * of each chunk, and `stream` waits for all three streams' work (after an
+ * error too, so the buffers are free once `stream` has been synchronised).
+ * Either way the host outputs are valid once `stream` has been synchronised,
+ * and they equal vidattn_fwd's bit for bit.  Host buffers
  * should be pinned for the copies to overlap.  h_seg_q/h_seg_kv and
  * d_seg_q/d_seg_kv follow the NULL rule of vidattn_fwd.
  */

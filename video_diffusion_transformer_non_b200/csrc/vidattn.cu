@@ -634,9 +634,14 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
       cudaEventDestroy(k_done);
     }
   }
-  // `stream` reaches this point only after the last copy-out
-  ok = ok && cudaEventRecord(done, cout) == cudaSuccess &&
-       cudaStreamWaitEvent(stream, done, 0) == cudaSuccess;
+  // `stream` waits for everything enqueued on the three side streams (a
+  // stream-wait takes the event's latest record), after an error too, so
+  // that the caller may free or reuse the buffers once `stream` is done
+  bool joined = true;
+  for (cudaStream_t side : {cin, cout, comp2})
+    joined = joined && cudaEventRecord(done, side) == cudaSuccess &&
+             cudaStreamWaitEvent(stream, done, 0) == cudaSuccess;
+  ok = ok && joined;
   cudaEventDestroy(start);
   cudaEventDestroy(done);
   if (!ok) return st != VIDATTN_OK ? st : VIDATTN_ERR_CUDA;
