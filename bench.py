@@ -67,8 +67,7 @@ def measured_traffic(w, summary=None, sources=KERNEL_SOURCES):
     kernel, or None when there is none or the kernel's code changed since
     (sha256 over its device sources with comments removed)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles",
-                        summary or f"vidattn_fwd_kernel_d{w.D}__{w.name}_h8.md")
+    path = os.path.join(ROOT, "profiles", summary or traffic_summary(w))
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -82,6 +81,12 @@ def measured_traffic(w, summary=None, sources=KERNEL_SOURCES):
         with open(os.path.join(csrc, f)) as fh:
             h.update(code_only(fh.read()).encode())
     return int(val.group(1)) if h.hexdigest() == sha.group(1) else None
+
+
+def traffic_summary(w, causal=False) -> str:
+    """Name of the committed ncu summary that holds the DRAM traffic of this
+    workload's attention launch (the causal limit has its own capture)."""
+    return f"vidattn_fwd_kernel_d{w.D}__{w.name}{'_causal' if causal else ''}_h8.md"
 
 
 def algorithmic_bytes(w) -> int:
@@ -482,7 +487,8 @@ def main(argv=None):
     achieved = flops_step / (kernel_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": UNIT,
                 "frac": achieved / peaks["bf16"],
-                "traffic": measured_traffic(w) if args.heads is None else None,
+                "traffic": (measured_traffic(w, traffic_summary(w, args.causal))
+                            if args.heads is None else None),
                 "peak_source": f"{peaks['source']} bf16 dense (burst)",
                 "frac_of_sustained": achieved / peaks["bf16_sustained"],
                 "kernel": f"vidattn_fwd_kernel<{w.D}>",

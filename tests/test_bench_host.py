@@ -73,6 +73,19 @@ def test_recorded_traffic_follows_the_code(tmp_path, monkeypatch):
 def test_committed_summaries_parse():
     """The committed ncu summaries carry both fields bench.py reads."""
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    for name in ("vidattn_fwd_kernel_d128__video_480p_h8.md", "rope3d_kernel_d128__video_480p.md"):
+    for name in ("vidattn_fwd_kernel_d128__video_480p_h8.md", "rope3d_kernel_d128__video_480p.md",
+                 "vidattn_fwd_kernel_d128__video_480p_causal_h8.md",
+                 "vidattn_fwd_kernel_d64__cogvideox_joint_h8.md"):
         text = open(os.path.join(root, "profiles", name)).read()
         assert "kernel_sources_sha256:" in text and "traffic_bytes_per_full_launch:" in text
+
+
+def test_causal_runs_read_the_causal_capture():
+    """A causal bench line takes its traffic from the causal capture, never
+    from the full-attention one of the same workload."""
+    w = wl.WORKLOADS["video_480p"]
+    assert bench.traffic_summary(w) == "vidattn_fwd_kernel_d128__video_480p_h8.md"
+    assert bench.traffic_summary(w, causal=True) == \
+        "vidattn_fwd_kernel_d128__video_480p_causal_h8.md"
+    assert bench.traffic_summary(wl.WORKLOADS["video_720p"], causal=True) != \
+        bench.traffic_summary(wl.WORKLOADS["video_720p"])
