@@ -7,8 +7,6 @@ count over every (query, key) pair of small workloads of the same kinds: ids
 compared token by token, the causal limit applied pair by pair, and for
 windows the nonzero entries of the oracle's probability matrix (the oracle's
 window rule is pinned on its own in test_window_oracle.py)."""
-import dataclasses
-
 import numpy as np
 import pytest
 
