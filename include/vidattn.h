@@ -87,8 +87,9 @@ typedef enum {
  * share scratch in flight.
  *
  * Errors: argument errors return their status before anything is enqueued;
- * launch failures return VIDATTN_ERR_CUDA.  S_q == 0 or B*H == 0 enqueues
- * nothing and returns VIDATTN_OK.  Kernel waits are bounded (2 s); a wait
+ * launch failures return VIDATTN_ERR_CUDA.  S_q == 0 (with the other
+ * arguments valid) enqueues nothing and returns VIDATTN_OK; B or H below 1
+ * is VIDATTN_ERR_BAD_SHAPE.  Kernel waits are bounded (2 s); a wait
  * that runs out sets a device error word that vidattn_device_status() reports.
  * While that word is set, the kernels of later calls on the device return at
  * once without writing their outputs, until vidattn_device_status() has
@@ -150,7 +151,9 @@ VIDATTN_API int vidattn_fwd_ex(const void* q, const void* k, const void* v,
  *
  *   win_t, win_h, win_w   odd, >= 1
  *   T, Hg, Wg             volume extents, 1..1024, 1..2048, 1..2048; every
- *                         coordinate must be below its extent
+ *                         coordinate must be below its extent (one that is
+ *                         not gives unspecified values for its rows; the
+ *                         coordinates are never used to address memory)
  *   S_kv                  <= 262144 (the key tiles of a CTA are listed in
  *                         shared memory)
  *   flags                 0 or VIDATTN_WINDOW_CLAMPED
@@ -262,7 +265,8 @@ VIDATTN_API int vidattn_fwd_noalloc(const void* q, const void* k, const void* v,
  *                Either the input itself (in place, contiguous input only)
  *                or a buffer that does not overlap it.
  *   k_in, k_out  both NULL to rotate q only.
- *   B, H >= 1, 2*B*H < 2^31;  D = 64 or 128.
+ *   B, H >= 1; n*B*H < 2^31 for n tensors (2 with k, 1 without);
+ *                D = 64 or 128.
  *   T, Hg, Wg >= 1; token_offset >= 0; token_offset + T*Hg*Wg <= S.
  *   theta        finite, > 0 (10000 in the common conventions).
  *   flags        0 or VIDATTN_ROPE_HALF_SPLIT.
