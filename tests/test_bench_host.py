@@ -90,3 +90,51 @@ def test_causal_runs_read_the_causal_capture():
         "vidattn_fwd_kernel_d128__video_480p_causal_h8.md"
     assert bench.traffic_summary(wl.WORKLOADS["video_720p"], causal=True) != \
         bench.traffic_summary(wl.WORKLOADS["video_720p"])
+
+
+def _run_bench(args, env_extra=None):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **(env_extra or {}))
+    p = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], cwd=root,
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.strip()]
+    return [json.loads(l) for l in lines]
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference`: one JSON line with the contract's keys,
+    the oracle timed on the host on the same workload and metric."""
+    (line,) = _run_bench(["--impl", "reference", "--workload", "joint_small", "--steps", "3",
+                          "--warmup", "3", "--ref-seconds", "3"])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["value"] > 0 and line["ms_per_step"] > 0
+    assert (line["steps"], line["warmup"], line["n_gpus"]) == (3, 3, 1)
+    assert line["higher_is_better"] is True and line["scaling"] == "weak"
+    assert line["vs_baseline"] is None and line["data"] == "synthetic"
+    assert line["config"]["workload"] == "joint_small"
+    cpu = line["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["value"] == line["value"] and cpu["cores"] >= 1
+    assert cpu["unit"] == bench.UNIT and "joint_small" in cpu["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT,
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under torchrun every rank but 0 exits at once without a line."""
+    assert _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "3",
+                       "--warmup", "3", "--ref-seconds", "1"],
+                      {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_bench_rejects_fewer_than_three_warmups():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    p = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--warmup", "2"],
+                       cwd=root, capture_output=True, text=True, timeout=120)
+    assert p.returncode != 0 and "warmup" in p.stderr
