@@ -25,6 +25,17 @@
  *
  * All entry points are C ABI, thread-safe for distinct streams, and never
  * throw.  Status codes are the vidattn_status values below.
+ *
+ * CUDA graphs: once set up, vidattn_fwd, vidattn_fwd_ex, vidattn_fwd_window,
+ * vidattn_fwd_noalloc and vidattn_rope3d enqueue kernel launches on `stream`
+ * and nothing else, so they can be captured into a graph.  Set-up happens on
+ * the first call on a device (kernel attributes, symbol addresses, occupancy
+ * queries: host calls only) and, for the calls that use scratch (ids or a
+ * window), on the first call on a stream or with a larger shape (cudaMalloc
+ * after synchronising that stream, which a capture does not allow).  So make
+ * one call of the largest shape on the capturing stream before capturing, or
+ * use vidattn_fwd_noalloc.  vidattn_fwd_host and vidattn_device_status are
+ * not for capture (events on library streams; a synchronisation).
  */
 #ifndef VIDATTN_H
 #define VIDATTN_H
