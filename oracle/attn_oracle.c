@@ -1,6 +1,7 @@
 /*
- * Test infrastructure only: the fp64 CPU oracle for segment-masked,
- * non-causal multi-head softmax attention.  Only the tests, the smoke check
+ * Test infrastructure only: the fp64 CPU oracle for segment-masked
+ * multi-head softmax attention (bidirectional, with an optional causal limit
+ * or 3D neighbourhood window, both described below).  Only the tests, the smoke check
  * and the benchmark's CPU-baseline leg load this file's library; the product
  * path never calls it, and it shares no code with the CUDA library.
  *
