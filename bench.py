@@ -304,6 +304,9 @@ def main(argv=None):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        ap.error(f"--gpus {args.gpus} but {world} rank(s) were launched: for N > 1 run "
+                 f"python -m torch.distributed.run --nproc-per-node N bench.py --gpus N")
     if args.impl == "reference":
         return run_reference(args, w, rank)
 

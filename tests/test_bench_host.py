@@ -124,17 +124,14 @@ def test_reference_arm_prints_the_contract_line():
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
-def test_reference_arm_runs_on_rank_zero_only():
-    """Under torchrun every rank but 0 exits at once without a line."""
-    assert _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "3",
-                       "--warmup", "3", "--ref-seconds", "1"],
-                      {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
-
-
-def test_bench_rejects_fewer_than_three_warmups():
+def test_bench_refuses_a_gpu_count_that_was_not_launched():
+    """--gpus N must match the ranks torchrun started; a lone process asked
+    for 2 GPUs stops with a message instead of timing one."""
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    p = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--warmup", "2"],
-                       cwd=root, capture_output=True, text=True, timeout=120)
-    assert p.returncode != 0 and "warmup" in p.stderr
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    p = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--impl", "reference"], cwd=root, env=env, capture_output=True,
+                       text=True, timeout=120)
+    assert p.returncode != 0 and "torch.distributed.run" in p.stderr

@@ -79,8 +79,8 @@ def test_reference_arm_rank0_prints_contract_line():
 
 
 def test_reference_arm_other_ranks_exit_without_work():
-    r = _run_bench(["--impl", "reference", "--workload", "video_720p", "--steps", "2",
-                    "--warmup", "3"], {"RANK": "1", "WORLD_SIZE": "2"})
+    r = _run_bench(["--impl", "reference", "--gpus", "2", "--workload", "video_720p",
+                    "--steps", "2", "--warmup", "3"], {"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0
     assert not [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
 
