@@ -4,10 +4,12 @@
 
 One step = one vidattn_fwd call (segment classification when ids are given,
 then the attention kernel) over one batch of the chosen workload, inputs
-already resident in HBM.  Default workload: video_480p (B1 H40 D128,
-S = 32760 tokens, one segment), a >=32k-token configuration of the kind the
->=60%-of-peak target is quoted on.  Its inputs (~1 GB per step) are larger
-than the 126 MB L2, so no flush is needed between steps.
+already resident in HBM.  Default workload: video_720p (B1 H24 D128,
+S = 119168 tokens: 118800 video, 256 text and 112 padding tokens in three
+segments), the largest single-GPU configuration and one of the >=32k-token
+configurations the >=60%-of-peak target is quoted on; video_480p and the
+others are reachable with --workload.  Its inputs (~2.2 GB per step) are
+larger than the 126 MB L2, so no flush is needed between steps.
 
 Under torchrun (N > 1) every rank runs its own replica (independent problem,
 seeded by rank): weak scaling, no collective on the data path.  Timing is on
@@ -100,7 +102,8 @@ def algorithmic_bytes(w) -> int:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    """nvidia-smi sampled every 20 ms while the timed region runs (read only:
+    no clock or power setting is touched)."""
     FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
               "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -116,7 +119,7 @@ class ClockSampler:
             self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=self.tmp, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
 
@@ -277,7 +280,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=150)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="video_480p")
+    ap.add_argument("--workload", default="video_720p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (smaller profiling cases)")
@@ -537,6 +540,10 @@ def main(argv=None):
             "rope3d": rope,
             "clocks": clocks,
         }
+        if clocks and clocks.get("sm_mhz"):
+            # the step's length in SM clock cycles at the median clock seen
+            # under load: comparable across runs whose clocks differ
+            clocks["mcycles_per_step"] = ms_per_step * 1e-3 * clocks["sm_mhz"]
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
