@@ -326,8 +326,13 @@ VIDATTN_API int vidattn_selftest_timeout(int timeout_us, vidattn_stream_t stream
 
 /* Frees the library's scratch buffers and destroys its internal streams (the
  * copy and second compute streams of vidattn_fwd_host) on every device, after
- * synchronising the streams concerned.  Call it while no other thread is
- * inside a vidattn call; later calls allocate again on demand. */
+ * synchronising the streams concerned, and forgets what it learnt about each
+ * device's CUDA context (symbol addresses, kernel attributes).  Call it while
+ * no other thread is inside a vidattn call; later calls set up and allocate
+ * again on demand.  Call it before cudaDeviceReset (or anything else that
+ * destroys a device's primary context) if the library is used again
+ * afterwards: without it the library would keep using addresses of the
+ * destroyed context. */
 VIDATTN_API void vidattn_release(void);
 
 /* Library version and the GPU architecture it was compiled for. */

@@ -4,16 +4,19 @@ after start-up, or code on a fixed memory budget).  Its segment summaries
 live in a fixed array inside the library instead of a buffer allocated on
 first use.
 
-The GPU test calls it through the C ABI twice in a row, with different shapes
-and segment layouts, and checks each result against the allocating entry
-point vidattn_fwd under the parity tolerances.  This file is collected last,
-so a run that stops at the first failure has already run every other test."""
-import ctypes
-
+The GPU test calls it through the C ABI several times in a row, with
+different shapes and segment layouts, through the same fixed array.  Each
+result must equal the allocating entry point vidattn_fwd's bit for bit (the
+same classifier and attention kernel run on the same summaries, only stored
+elsewhere) and match the fp64 oracle under the parity tolerances.  One case
+has two samples with different ids, so a wrong per-sample offset into the
+array would show.  This file is collected last, so a run that stops at the
+first failure has already run every other test."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from video_diffusion_transformer_non_b200 import binding
 from video_diffusion_transformer_non_b200 import workloads as wl
 
@@ -21,12 +24,11 @@ TOL_MAX_OUT, TOL_MEAN_OUT, TOL_LSE = 2e-2, 2e-3, 1e-3
 SCRATCH_LIMIT = 9
 
 
-def _dev_case(B, H, runs, D, seed):
-    seg = wl.segment_ids(runs, B)
+def _case(B, H, seg, D, seed):
     S = seg.shape[1]
     c = wl.make_random(B, H, S, S, D, seed, seg, seg.copy())
     up = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
-    return dict(q=up(c["q"]), k=up(c["k"]), v=up(c["v"]),
+    return dict(host=c, q=up(c["q"]), k=up(c["k"]), v=up(c["v"]),
                 sq=torch.from_numpy(seg.copy()).cuda(), sk=torch.from_numpy(seg.copy()).cuda(),
                 B=B, H=H, S=S, D=D, scale=c["scale"])
 
@@ -43,21 +45,43 @@ def _run(fn, c):
     return out, lse
 
 
+def _against_oracle(c, out, lse):
+    h = c["host"]
+    ro, rl = oracle.attn_fwd(h["q"], h["k"], h["v"], h["seg_q"], h["seg_kv"], h["scale"])
+    og = out.double().cpu().numpy()
+    lg = lse.double().cpu().numpy()
+    empty = np.isneginf(rl)
+    assert np.array_equal(np.isneginf(lg), empty)
+    assert np.all(og[empty] == 0.0)
+    d = np.abs(og[~empty] - ro[~empty])
+    assert d.max() <= TOL_MAX_OUT and d.mean() <= TOL_MEAN_OUT, (d.max(), d.mean())
+    assert np.abs(lg[~empty] - rl[~empty]).max() <= TOL_LSE
+
+
 @pytest.mark.gpu
-def test_no_alloc_matches_allocating_entry_point_on_two_calls():
+def test_no_alloc_matches_allocating_entry_point_on_calls_in_a_row():
     binding.load_library()
-    cases = [_dev_case(2, 3, ((700, 0), (140, 1), (37, 2)), 128, 71),
-             _dev_case(1, 2, ((300, 5), (29, 6), (200, 5), (16, 9)), 64, 72)]
-    for c in cases:                       # two calls in a row through the same scratch
+    # two samples with different ids (the second sample's summaries sit
+    # B * ceil(S/128) entries further into the fixed array than the first's)
+    ids0 = np.concatenate([np.full(700, 0), np.full(140, 1), np.full(37, 2)])
+    ids1 = np.concatenate([np.full(300, 4), np.full(450, 0), np.full(90, 2), np.full(37, 9)])
+    per_sample = np.stack([ids0, ids1]).astype(np.int32)
+    cases = [_case(2, 3, per_sample, 128, 71),
+             _case(1, 2, wl.segment_ids(((300, 5), (29, 6), (200, 5), (16, 9)), 1), 64, 72),
+             _case(2, 2, wl.segment_ids(((1500, 0), (260, 1), (40, 2)), 2), 128, 73)]
+    first = None
+    for c in cases + cases[:1]:           # calls in a row through the same array, then again
         out_n, lse_n = _run(binding.vidattn_fwd_noalloc, c)
         out_r, lse_r = _run(binding.vidattn_fwd, c)
-        assert not bool(torch.isnan(out_n.float()).any()) and not bool(torch.isnan(lse_n).any())
-        empty = torch.isneginf(lse_r)
-        assert torch.equal(torch.isneginf(lse_n), empty)
-        d = (out_n.double() - out_r.double()).abs()
-        assert float(d.max()) <= TOL_MAX_OUT and float(d.mean()) <= TOL_MEAN_OUT
-        dl = (lse_n.double() - lse_r.double()).abs()[~empty]
-        assert dl.numel() == 0 or float(dl.max()) <= TOL_LSE
+        assert torch.equal(out_n.view(torch.int16), out_r.view(torch.int16))
+        assert torch.equal(lse_n.view(torch.int32), lse_r.view(torch.int32))
+        _against_oracle(c, out_n, lse_n)
+        if first is None:
+            first = (out_n.clone(), lse_n.clone())
+    # the repeated first case equals its first result: nothing left in the
+    # array by the calls in between is read
+    assert torch.equal(out_n.view(torch.int16), first[0].view(torch.int16))
+    assert torch.equal(lse_n.view(torch.int32), first[1].view(torch.int32))
 
 
 def test_no_alloc_rejects_shapes_beyond_its_scratch():

@@ -794,10 +794,6 @@ VIDATTN_API void vidattn_release(void) {
       }
     }
   }
-  if (g_scratch.empty()) {
-    cudaSetDevice(prev);
-    return;
-  }
   for (auto& kv : g_scratch) {
     if (kv.second.ptr) {
       cudaSetDevice(kv.first.first);
@@ -806,6 +802,12 @@ VIDATTN_API void vidattn_release(void) {
     }
   }
   g_scratch.clear();
+  // Per-context state: the symbol addresses (device error word, the
+  // no-allocation array), kernel attributes and occupancy results are looked
+  // up again by the next call, so a context created after this (say, after
+  // cudaDeviceReset) never sees addresses of the old one.
+  g_devices.clear();
+  g_noalloc_ptr.clear();
   cudaSetDevice(prev);
 }
 
