@@ -1,7 +1,13 @@
 """Sequence-parallel (Ulysses) attention: the all_to_all layout changes around
 the attention call.  CPU: world size 2 and 4 with gloo, the fp64 oracle as the
-per-shard attention, compared with the oracle on the whole sequence.  GPU: a
-world of one over NCCL through the CUDA kernel, compared with vidattn_fwd."""
+per-shard attention, compared with the oracle on the whole sequence.  GPU:
+(a) a world of one over NCCL through the CUDA kernel, compared with the
+direct calls bit for bit and with the fp64 oracle under the parity
+tolerances; (b) world size 2 as two processes exchanging over gloo, each
+running its head shard's attention (and rotation) with the CUDA kernels on
+the one GPU (independent launches: no kernel waits on another process),
+compared with the fp64 oracle over the whole sequence, for B = 1 (the
+exchange lands in the result directly) and B = 2 (through a buffer)."""
 import os
 import socket
 import sys
@@ -107,11 +113,18 @@ def test_ulysses_single_gpu_world_equals_kernel():
         up = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
         q, k, v = up(c["q"]), up(c["k"]), up(c["v"])
         sg = torch.from_numpy(seg.copy()).cuda()
-        o1, l1 = ulysses_attention(q, k, v, sg, c["scale"], n_chunks=2)
-        o2, l2 = binding.attention(q, k, v, sg, sg, c["scale"])
-        torch.cuda.synchronize()
-        assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
-        assert torch.equal(l1, l2)
+        import oracle
+        from _gpu_helpers import compare
+        for causal in (False, True):
+            o1, l1 = ulysses_attention(q, k, v, sg, c["scale"], causal=causal, n_chunks=2)
+            o2, l2 = binding.attention(q, k, v, sg, sg, c["scale"], causal=causal)
+            torch.cuda.synchronize()
+            assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+            assert torch.equal(l1, l2)
+            ro, rl = oracle.attn_fwd(c["q"], c["k"], c["v"], seg, seg.copy(), c["scale"],
+                                     causal=causal)
+            compare(o1.double().cpu().numpy(), l1.double().cpu().numpy(), ro, rl,
+                    f"ulysses world 1, causal={causal}")
     finally:
         dist.destroy_process_group()
 
@@ -229,5 +242,135 @@ def test_ulysses_single_gpu_window_with_rope_equals_direct_calls():
         torch.cuda.synchronize()
         assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
         assert torch.equal(l1, l2)
+        # against the oracle: fp64 rotation rounded to bf16, then the window rule
+        import oracle
+        from oracle.rope3d import rope3d_f64
+        from _gpu_helpers import compare
+        rot = lambda x: wl.f32_to_bf16_bits(rope3d_f64(x, grid, bands).astype(np.float32))
+        coords = wl.raster_coords(grid, B)
+        win = dict(coord_q=coords, coord_kv=coords.copy(), size=(3, 5, 5), extent=grid,
+                   clamped=True)
+        ro, rl = oracle.attn_fwd(rot(c["q"]), rot(c["k"]), c["v"], scale=c["scale"], window=win)
+        compare(o1.double().cpu().numpy(), l1.double().cpu().numpy(), ro, rl,
+                "ulysses world 1, window + rope")
     finally:
         dist.destroy_process_group()
+
+
+# --------------------------------------------- world 2 over gloo, CUDA per rank
+
+def _to_gpu_bf16(t):
+    """bf16 bit patterns carried in a float16-typed CPU tensor -> bf16 on cuda:0."""
+    return t.contiguous().view(torch.bfloat16).cuda()
+
+
+def _from_gpu_bf16(t):
+    return t.cpu().view(torch.float16)
+
+
+def _cuda_attn_gloo(q, k, v, seg_q, seg_kv, scale, causal, window=None):
+    """A rank's head-shard attention with the CUDA kernel; the exchange around
+    it stays on the CPU (gloo), in float16-typed tensors holding bf16 bits."""
+    from video_diffusion_transformer_non_b200 import binding
+    qd, kd, vd = _to_gpu_bf16(q), _to_gpu_bf16(k), _to_gpu_bf16(v)
+    if window is not None:
+        co = window["coords"].cuda()
+        o, l = binding.attention_window(qd, kd, vd, co, co, window["size"], window["extent"],
+                                        window["clamped"], scale)
+    else:
+        sq = None if seg_q is None else seg_q.cuda()
+        o, l = binding.attention(qd, kd, vd, sq, sq, scale, causal=causal)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    return _from_gpu_bf16(o), l.cpu()
+
+
+def _cuda_rope_gloo(q, k, rope):
+    from video_diffusion_transformer_non_b200 import binding
+    qr, kr = binding.rope3d(_to_gpu_bf16(q), _to_gpu_bf16(k), rope["grid"], rope["bands"],
+                            theta=rope.get("theta", 10000.0))
+    torch.cuda.synchronize()
+    return _from_gpu_bf16(qr), _from_gpu_bf16(kr)
+
+
+def _rank_main_cuda(rank, world, port, case, coords, opts, q_out):
+    import torch.distributed as dist
+    from video_diffusion_transformer_non_b200.ulysses import ulysses_attention
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        S = case["q"].shape[2]
+        Sl = S // world
+        sl = slice(rank * Sl, (rank + 1) * Sl)
+        shard = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, :, sl]).view(np.float16))
+        seg = None if case["seg_q"] is None else torch.from_numpy(
+            np.ascontiguousarray(case["seg_q"][:, sl]))
+        win = None
+        if opts.get("window") is not None:
+            win = dict(opts["window"], coords=torch.from_numpy(np.ascontiguousarray(coords[:, sl])))
+        out, lse = ulysses_attention(shard(case["q"]), shard(case["k"]), shard(case["v"]), seg,
+                                     case["scale"], opts.get("causal", False), None,
+                                     opts["n_chunks"], _cuda_attn_gloo, window=win,
+                                     rope=opts.get("rope"), rope_fn=_cuda_rope_gloo)
+        q_out.put((rank, out.view(torch.bfloat16).double().numpy(), lse.double().numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run_world(world, case, coords, opts):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_cuda, args=(r, world, port, case, coords, opts, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=300) for _ in range(world)], key=lambda x: x[0])
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    return (np.concatenate([r[1] for r in res], axis=2),
+            np.concatenate([r[2] for r in res], axis=2))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,causal", [(1, False), (2, True)])
+def test_ulysses_world2_cuda_attention_matches_oracle(B, causal):
+    """Two ranks exchange over gloo; each runs its head shard on the GPU with
+    the CUDA kernel (ids, optionally the causal limit, two head chunks); the
+    gathered shards match the fp64 oracle over the whole sequence."""
+    import oracle
+    from _gpu_helpers import compare
+    from video_diffusion_transformer_non_b200 import workloads as wl
+    H, D = 8, 128
+    seg = wl.segment_ids(((900, 0), (200, 1), (100, 2)), B)
+    S = seg.shape[1]
+    case = wl.make_random(B, H, S, S, D, 64, seg, seg.copy())
+    out, lse = _run_world(2, case, None, dict(n_chunks=2, causal=causal))
+    ro, rl = oracle.attn_fwd(case["q"], case["k"], case["v"], seg, seg.copy(), case["scale"],
+                             causal=causal)
+    compare(out, lse, ro, rl, f"ulysses world 2 (gloo), CUDA attention, B={B}")
+
+
+@pytest.mark.gpu
+def test_ulysses_world2_cuda_window_with_rope_matches_oracle():
+    """The same with the 3D RoPE pass (global positions) and a clamped 3D
+    neighbourhood window, both on the GPU per rank."""
+    import oracle
+    from oracle.rope3d import rope3d_f64
+    from _gpu_helpers import compare
+    from video_diffusion_transformer_non_b200 import workloads as wl
+    grid, bands = (4, 8, 20), (44, 42, 42)
+    B, H, D = 1, 4, 128
+    S = int(np.prod(grid))
+    case = wl.make_random(B, H, S, S, D, 65)
+    coords = wl.raster_coords(grid, B)
+    window = dict(size=(3, 5, 5), extent=grid, clamped=True)
+    out, lse = _run_world(2, case, coords, dict(n_chunks=2, window=window,
+                                                rope=dict(grid=grid, bands=bands)))
+    rot = lambda x: wl.f32_to_bf16_bits(rope3d_f64(x, grid, bands).astype(np.float32))
+    win = dict(coord_q=coords, coord_kv=coords.copy(), size=(3, 5, 5), extent=grid, clamped=True)
+    ro, rl = oracle.attn_fwd(rot(case["q"]), rot(case["k"]), case["v"], scale=case["scale"],
+                             window=win)
+    compare(out, lse, ro, rl, "ulysses world 2 (gloo), CUDA window + rope")

@@ -39,41 +39,77 @@ def _world(group):
 
 
 class _Exchange:
-    """One all_to_all in flight and the reshaping that follows it."""
+    """One all_to_all in flight and the layout change that follows it.
 
-    def __init__(self, send, finish, P, group):
-        self.recv = torch.empty_like(send)
-        self.finish = finish
-        self.work = dist.all_to_all_single(self.recv, send, group=group, async_op=True) \
-            if P > 1 else None
-        if P == 1:
-            self.recv = send
+    `send` is contiguous with the destination rank outermost.  `recv` is
+    where the collective lands (it may be the caller's final buffer, then
+    `finish` is None and nothing is copied afterwards); `finish(recv)` makes
+    the final layout (at most one copy)."""
+
+    def __init__(self, send, recv, finish, P, group):
+        self.recv, self.finish = recv, finish
+        self.work = None
+        if P > 1:
+            self.work = dist.all_to_all_single(recv, send, group=group, async_op=True)
+        elif recv.data_ptr() != send.data_ptr():
+            recv.copy_(send)
 
     def result(self):
         if self.work is not None:
             self.work.wait()
-        return self.finish(self.recv)
+        return self.recv if self.finish is None else self.finish(self.recv)
 
 
 def _seq_to_heads(x: torch.Tensor, P: int, group) -> _Exchange:
-    """[B, H, Sl, *r] sequence shard -> [B, H/P, P*Sl, *r] head shard."""
+    """[B, H, Sl, *r] sequence shard -> [B, H/P, P*Sl, *r] head shard.
+
+    Copies: the send side is a view of x when B == 1 and x is contiguous (the
+    rank-major order is then x's own), else one copy; the receive side is one
+    copy, recv [P, B, H/P, Sl] -> [B, H/P, P, Sl], into the result."""
     B, H, Sl = x.shape[:3]
-    rest = x.shape[3:]
-    send = x.reshape(B, P, H // P, Sl, *rest).movedim(1, 0).contiguous()
-    # recv[p] = this rank's heads from sequence shard p
-    return _Exchange(send, lambda r: r.movedim(0, 2).reshape(B, H // P, P * Sl, *rest)
-                     .contiguous(), P, group)
+    rest = tuple(x.shape[3:])
+    Hp = H // P
+    send = x.reshape(B, P, Hp, Sl, *rest).movedim(1, 0)
+    if not send.is_contiguous():
+        send = send.contiguous()
+    if P == 1:
+        # nothing moves: the head shard is the sequence shard
+        return _Exchange(send, send, lambda r: r.reshape(B, H, Sl, *rest), P, group)
+    recv = torch.empty_like(send)
+
+    def finish(r):
+        out = torch.empty((B, Hp, P * Sl, *rest), dtype=x.dtype, device=x.device)
+        # recv[p] = this rank's heads of sequence shard p
+        out.view(B, Hp, P, Sl, *rest).copy_(r.permute(1, 2, 0, *range(3, 4 + len(rest))))
+        return out
+
+    return _Exchange(send, recv, finish, P, group)
 
 
-def _heads_to_seq(y: torch.Tensor, P: int, group) -> _Exchange:
-    """[B, H/P, S, *r] head shard -> [B, H, S/P, *r] sequence shard."""
+def _heads_to_seq(y: torch.Tensor, P: int, group, dst: torch.Tensor) -> _Exchange:
+    """[B, H/P, S, *r] head shard -> dst [B, H, S/P, *r] sequence shard.
+
+    Copies: the send side is one copy, y [B, H/P, P, Sl] -> [P, B, H/P, Sl];
+    the collective lands in dst directly when B == 1 (the receive order,
+    source rank = head group outermost, is then dst's own), else in a buffer
+    copied into dst once."""
     B, Hl, S = y.shape[:3]
-    rest = y.shape[3:]
+    rest = tuple(y.shape[3:])
     Sl = S // P
-    send = y.reshape(B, Hl, P, Sl, *rest).movedim(2, 0).contiguous()
-    # recv[p] = this rank's sequence shard for head group p
-    return _Exchange(send, lambda r: r.movedim(0, 1).reshape(B, P * Hl, Sl, *rest)
-                     .contiguous(), P, group)
+    send = y.reshape(B, Hl, P, Sl, *rest).movedim(2, 0)
+    if not send.is_contiguous():
+        send = send.contiguous()
+    direct = dst.reshape(B, P, Hl, Sl, *rest).movedim(1, 0)   # dst in receive order
+    if direct.is_contiguous():
+        return _Exchange(send, direct, None, P, group)
+    recv = torch.empty_like(send)
+
+    def finish(r):
+        # recv[p] = this rank's sequence shard of head group p
+        dst.view(B, P, Hl, Sl, *rest).copy_(r.movedim(0, 1))
+        return dst
+
+    return _Exchange(send, recv, finish, P, group)
 
 
 def _cuda_attention(q, k, v, seg_q, seg_kv, scale, causal, window=None):
@@ -134,7 +170,10 @@ def ulysses_attention(q, k, v, seg=None, scale=None, causal=False, group=None, n
     for c in range(n_chunks):          # every input exchange goes out first
         hs = slice(c * Hc, (c + 1) * Hc)
         inputs.append([_seq_to_heads(t[:, hs], P, group) for t in (q, k, v)])
-    outputs = []
+    # the results land in out and lse (allocated as the attention's results
+    # are typed), chunk c in heads [c Hc, (c+1) Hc)
+    out = lse = None
+    pending = []
     for c in range(n_chunks):
         qh, kh, vh = (x.result() for x in inputs[c])
         if rope is not None:
@@ -143,7 +182,11 @@ def ulysses_attention(q, k, v, seg=None, scale=None, causal=False, group=None, n
             o, l = attn(qh, kh, vh, None, None, scale, False, window=win_full)
         else:
             o, l = attn(qh, kh, vh, seg_full, seg_full, scale, causal)
-        outputs.append((_heads_to_seq(o, P, group), _heads_to_seq(l, P, group)))
-    outs = [o.result() for o, _ in outputs]
-    lses = [l.result() for _, l in outputs]
-    return torch.cat(outs, dim=1), torch.cat(lses, dim=1)
+        if out is None:
+            out = torch.empty((B, H, Sl, D), dtype=o.dtype, device=o.device)
+            lse = torch.empty((B, H, Sl), dtype=l.dtype, device=l.device)
+        hs = slice(c * Hc, (c + 1) * Hc)
+        pending += [_heads_to_seq(o, P, group, out[:, hs]), _heads_to_seq(l, P, group, lse[:, hs])]
+    for x in pending:
+        x.result()
+    return out, lse
