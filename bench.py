@@ -293,6 +293,8 @@ def main(argv=None):
     ap.add_argument("--rope", action="store_true",
                     help="each step rotates q and k (vidattn_rope3d, the workload's 3D RoPE "
                          "convention) before the attention")
+    ap.add_argument("--split", type=int, default=0,
+                    help="key splits per query block (VIDATTN_SPLIT_KV); 0: the library's choice")
     ap.add_argument("--rope-half-split", action="store_true",
                     help="with --rope: pair features k and k + d/2 instead of 2k and 2k+1")
     args = ap.parse_args(argv)
@@ -349,7 +351,7 @@ def main(argv=None):
         ck = torch.from_numpy(win["coord_kv"].copy()).to(dev)
         win_flags = binding.VIDATTN_WINDOW_CLAMPED if w.window_clamped else 0
 
-    flags = binding.VIDATTN_CAUSAL if args.causal else 0
+    flags = (binding.VIDATTN_CAUSAL if args.causal else 0) | binding.VIDATTN_SPLIT_KV(args.split)
     use_rope = args.rope
     rope_interleaved = w.rope_interleaved and not args.rope_half_split
     # the attention reads the rotated q and k when the step includes the rotation
@@ -536,7 +538,11 @@ def main(argv=None):
             "hbm_gbs": algorithmic_bytes(w) / (kernel_ms * 1e-3) / 1e9,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (binding.kernels_per_call(
-                sq, sk, w.B, w.H, w.S_q, w.S_kv, w.D) + (1 if use_rope or windowed else 0)),
+                sq, sk, w.B, w.H, w.S_q, w.S_kv, w.D, flags) + (1 if use_rope or windowed else 0)),
+            "launch": {"grid_ctas": min(148, w.B * w.H * -(-w.S_q // 256) * binding.split_count(
+                           sq, w.B, w.H, w.S_q, w.S_kv, flags)),
+                       "key_splits": binding.split_count(sq, w.B, w.H, w.S_q, w.S_kv, flags),
+                       "persistent": True},
             "rope3d": rope,
             "clocks": clocks,
         }

@@ -115,6 +115,10 @@ VIDATTN_API int vidattn_fwd(const void* q, const void* k, const void* v,
 
 /* Flags of vidattn_fwd_ex. */
 #define VIDATTN_CAUSAL 1   /* key j visible to query i only if also j <= i + (S_kv - S_q) */
+/* Split each 256-row query block's keys into n ranges (1 <= n <= 64), run
+ * as separate work units and merged by a second kernel; 0 (the default)
+ * lets the library choose (vidattn_split_count). */
+#define VIDATTN_SPLIT_KV(n) (((n) & 0xFF) << 8)
 
 /*
  * vidattn_fwd_ex — vidattn_fwd with options.  flags = 0 is exactly
@@ -125,8 +129,12 @@ VIDATTN_API int vidattn_fwd(const void* q, const void* k, const void* v,
  * paragraph, combines with full-attention generation in one backbone;
  * combined with segment ids this is block-diagonal causal attention).  Key
  * tiles past the limit are never loaded.  Rows that see no key give out = 0,
- * lse = -inf.  Unknown flag bits return VIDATTN_ERR_BAD_SHAPE.  Other
- * arguments, errors and ownership: as vidattn_fwd.
+ * lse = -inf.  flags may also carry VIDATTN_SPLIT_KV(n) (a split count
+ * above 64 is VIDATTN_ERR_BAD_SHAPE): the same result within rounding (the
+ * ranges' partials are merged in fp32), for callers that know their
+ * launch shape better than vidattn_split_count.  Unknown flag bits return
+ * VIDATTN_ERR_BAD_SHAPE.  Other arguments, errors and ownership: as
+ * vidattn_fwd; the scratch also holds a split launch's partials.
  */
 VIDATTN_API int vidattn_fwd_ex(const void* q, const void* k, const void* v,
                                const int32_t* seg_q, const int32_t* seg_kv,
@@ -222,8 +230,11 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
  * fixed device-memory budget, for whom the on-demand scratch of vidattn_fwd
  * (a cudaMalloc on first use) is not allowed.
  *
- * Same arguments, layouts and results as vidattn_fwd; the caller still
- * passes every input and output.  The library allocates nothing: the segment
+ * Same arguments and layouts as vidattn_fwd; the caller still passes every
+ * input and output.  It never splits the keys (a split launch keeps partial
+ * results in scratch), so its results equal, bit for bit, those of
+ * vidattn_fwd_ex with VIDATTN_SPLIT_KV(1), and those of vidattn_fwd whenever
+ * vidattn_split_count() is 1.  The library allocates nothing: the segment
  * summaries use a fixed array in the library's device memory (512 KiB on every
  * GPU that loads the library, held until the process exits).  Limit, when
  * segment ids are given: B * (ceil(S_q/128) + ceil(S_kv/128)) <= 32768 (for
@@ -310,11 +321,30 @@ VIDATTN_API const char* vidattn_status_string(int status);
  * VIDATTN_OK. */
 VIDATTN_API int vidattn_device_status(vidattn_stream_t stream);
 
-/* Number of kernels one vidattn_fwd call with these arguments launches
- * (0 when there is nothing to compute; 2 with segment ids; 1 without).
+/* Launch heuristic: the number of key splits a vidattn_fwd_ex call with
+ * these arguments uses (flags as for vidattn_fwd_ex; 0 when there is nothing
+ * to compute or the flags are invalid).  The attention kernel works on units
+ * of (b, h, 256 query rows), longest first under the causal limit: one CTA
+ * per unit, or, at D = 128 with more units than SMs and at most 64 key tiles
+ * (short units, whose epilogues then overlap the next unit's loads),
+ * persistent with one CTA per SM looping over units.  When a call
+ * has fewer than 74 such units (half of the B200's 148 SMs) the library
+ * splits every unit's key tiles into ceil(148 / units) ranges (at most 16,
+ * at least 8 key tiles each: shorter ranges cost more in the merge than they
+ * gain), unless VIDATTN_SPLIT_KV asks for a number;
+ * each range is a unit of its own, and a second kernel merges the ranges'
+ * partial results (O / l and log-sum-exp per row, fp32, in the library's
+ * scratch: 4 * (D + 1) bytes per row, head and split).  With segment ids and
+ * more than 2048 key tiles nothing is split.  Pure host logic; no CUDA call. */
+VIDATTN_API int vidattn_split_count(const int32_t* seg_q, int B, int H, int S_q, int S_kv,
+                                    int flags);
+
+/* Number of kernels one vidattn_fwd_ex call with these arguments launches
+ * (0 when there is nothing to compute): the attention kernel, plus the tile
+ * classifier with segment ids, plus the merge of a split launch.
  * Pure host logic; no CUDA call. */
 VIDATTN_API int vidattn_kernels_per_call(const int32_t* seg_q, const int32_t* seg_kv,
-                                         int B, int H, int S_q, int S_kv, int D);
+                                         int B, int H, int S_q, int S_kv, int D, int flags);
 
 /* Failure-detection self-test: enqueues a one-warp kernel that waits, with the
  * attention kernel's own bounded wait, on an mbarrier that nothing arrives on.

@@ -58,8 +58,9 @@ class Guarded:
         assert not bool(torch.isnan(self.lse).any()), "some lse element was never written"
 
 
-def run_gpu(case, scale=None, check=True, causal=False):
-    """case: dict of numpy inputs (q, k, v bf16 bits; seg_q, seg_kv int32 or None)."""
+def run_gpu(case, scale=None, check=True, causal=False, flags=0):
+    """case: dict of numpy inputs (q, k, v bf16 bits; seg_q, seg_kv int32 or None).
+    flags: extra vidattn_fwd_ex flags (a VIDATTN_SPLIT_KV request)."""
     q, k, v = (to_dev_bf16(case[n]) for n in ("q", "k", "v"))
     sq, sk = to_dev_i32(case.get("seg_q")), to_dev_i32(case.get("seg_kv"))
     B, H, S_q, D = case["q"].shape
@@ -67,7 +68,7 @@ def run_gpu(case, scale=None, check=True, causal=False):
     g = Guarded(B, H, S_q, D)
     sc = case["scale"] if scale is None else scale
     st = binding.vidattn_fwd_ex(q, k, v, sq, sk, g.out, g.lse, B, H, S_q, S_kv, D, sc,
-                                binding.VIDATTN_CAUSAL if causal else 0)
+                                (binding.VIDATTN_CAUSAL if causal else 0) | flags)
     assert st == 0, binding.status_string(st)
     torch.cuda.synchronize()
     assert binding.device_status() == 0
@@ -94,8 +95,8 @@ def compare(out_gpu, lse_gpu, out_ref, lse_ref, what=""):
     return {}
 
 
-def check_all_rows(case, scale=None, what="", causal=False):
-    out, lse = run_gpu(case, scale, causal=causal)
+def check_all_rows(case, scale=None, what="", causal=False, flags=0):
+    out, lse = run_gpu(case, scale, causal=causal, flags=flags)
     ro, rl = oracle.attn_fwd(case["q"], case["k"], case["v"], case.get("seg_q"),
                              case.get("seg_kv"), case["scale"] if scale is None else scale,
                              causal=causal)

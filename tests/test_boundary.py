@@ -102,9 +102,39 @@ def test_host_entry_point_argument_errors(lib):
 
 
 def test_kernels_per_call(lib):
+    # tiny: 4 units of 256 query rows, but only 4 key tiles: no split
     assert binding.kernels_per_call(None, None, 1, 2, 512, 512, 64) == 1
-    assert binding.kernels_per_call(A, A, 2, 12, 4389, 4389, 128) == 2
+    assert binding.kernels_per_call(A, A, 2, 12, 4389, 4389, 128) == 2      # classify + attention
+    assert binding.kernels_per_call(None, None, 1, 40, 32760, 32760, 128) == 1
+    assert binding.kernels_per_call(A, A, 1, 2, 512, 8192, 64) == 3         # + classify + merge
+    assert binding.kernels_per_call(None, None, 1, 40, 32760, 32760, 128,
+                                    binding.VIDATTN_SPLIT_KV(2)) == 2
     assert binding.kernels_per_call(None, None, 1, 2, 0, 512, 64) == 0
+
+
+def test_split_heuristic(lib):
+    """The launch heuristic (pure host logic): key splits only when the
+    256-row query blocks x heads x batch are fewer than 74 (half of 148 SMs),
+    ceil(148 / units) of them, at most 16 and at least 8 key tiles each; the
+    VIDATTN_SPLIT_KV request overrides it; nothing with ids beyond 2048 key
+    tiles (the summaries are walked in global memory there)."""
+    sc = binding.split_count
+    S = binding.VIDATTN_SPLIT_KV
+    assert sc(None, 1, 2, 512, 512) == 1              # tiny: 4 key tiles, too short to split
+    assert sc(None, 1, 2, 512, 100000) == 16          # 4 units, many key tiles: capped at 16
+    assert sc(None, 1, 1, 256, 128 * 15) == 1         # 15 key tiles: one range of 8+
+    assert sc(None, 1, 1, 256, 128 * 16) == 2
+    assert sc(None, 1, 2, 512, 128 * 40) == 5         # 4 units, 40 key tiles: 8 each
+    assert sc(None, 1, 36, 512, 4096) == 3            # 72 units: ceil(148 / 72)
+    assert sc(None, 1, 37, 512, 4096) == 1            # 74 units: enough
+    assert sc(A, 2, 12, 4389, 4389) == 1              # joint_small: 432 units
+    assert sc(None, 1, 40, 32760, 32760) == 1
+    assert sc(None, 1, 1, 256, 300000) == 16          # no ids: any length splits
+    assert sc(A, 1, 1, 256, 300000) == 1              # ids beyond 2048 key tiles: never
+    assert sc(None, 1, 40, 32760, 32760, S(5)) == 5   # a request wins
+    assert sc(None, 1, 2, 512, 512, S(64)) == 64
+    assert sc(None, 1, 2, 512, 512, S(65)) == 0       # above 64: invalid
+    assert sc(None, 1, 2, 0, 512) == 0 and sc(None, 1, 2, 512, 0) == 1
 
 
 def test_selftest_argument_range(lib):

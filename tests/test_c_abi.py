@@ -22,7 +22,8 @@ int main(void) {
   const char* v = vidattn_version();
   if (!v || !strstr(v, "sm_100a")) return 1;
   if (strcmp(vidattn_status_string(VIDATTN_OK), "ok") != 0) return 2;
-  if (vidattn_kernels_per_call(NULL, NULL, 1, 2, 512, 512, 64) != 1) return 3;
+  if (vidattn_kernels_per_call(NULL, NULL, 1, 2, 512, 512, 64, 0) != 1) return 3;
+  if (vidattn_split_count(NULL, 1, 40, 32760, 32760, VIDATTN_SPLIT_KV(3)) != 3) return 3;
   /* argument errors, returned before anything touches a device */
   if (vidattn_fwd(NULL, NULL, NULL, NULL, NULL, NULL, NULL, 1, 2, 256, 256, 128, 0.1f, NULL)
       != VIDATTN_ERR_NULL) return 4;

@@ -22,14 +22,80 @@ pytestmark = pytest.mark.gpu
 
 # ------------------------------------------------------------ shapes, no ids
 
+@pytest.mark.parametrize("n_split", [0, 1])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("B,H,S_q,S_kv", [
     (1, 1, 1, 1), (1, 2, 128, 128), (1, 2, 127, 129), (2, 2, 129, 127),
     (1, 3, 300, 77), (1, 2, 256, 1000), (2, 1, 513, 384), (1, 1, 640, 2053),
 ])
-def test_shapes_single_segment(B, H, S_q, S_kv, D):
+def test_shapes_single_segment(B, H, S_q, S_kv, D, n_split):
+    """n_split 0: the launch's own choice (these short calls mostly split
+    their keys); 1: no split, every key tile of a query block in one unit."""
     c = wl.make_random(B, H, S_q, S_kv, D, seed=S_q * 7 + S_kv + D)
-    check_all_rows(c, what=f"B{B} H{H} Sq{S_q} Skv{S_kv} D{D}")
+    check_all_rows(c, what=f"B{B} H{H} Sq{S_q} Skv{S_kv} D{D} split {n_split}",
+                   flags=binding.VIDATTN_SPLIT_KV(n_split))
+
+
+# ------------------------------------------------------------- key splits
+# The launch splits each 256-row query block's keys into ranges when a call
+# has few query blocks (vidattn_split_count); VIDATTN_SPLIT_KV(n) forces n.
+# Every count must give the oracle's result: splits with no key, splits of
+# one tile, ids whose rows see no key of a split, the causal limit.
+
+@pytest.mark.parametrize("n_split", [1, 2, 3, 5, 8, 64])
+@pytest.mark.parametrize("D", [64, 128])
+def test_key_splits_single_segment(n_split, D):
+    c = wl.make_random(1, 2, 640, 1100, D, seed=900 + n_split + D)
+    check_all_rows(c, what=f"split {n_split} D{D}", flags=binding.VIDATTN_SPLIT_KV(n_split))
+
+
+@pytest.mark.parametrize("n_split", [1, 2, 7])
+def test_key_splits_with_ids(n_split):
+    c = runs_case(2, 3, ((700, 0), (140, 1), (37, 2)), 128, 34)
+    check_all_rows(c, what=f"ids, split {n_split}", flags=binding.VIDATTN_SPLIT_KV(n_split))
+
+
+@pytest.mark.parametrize("n_split", [1, 3])
+def test_key_splits_causal(n_split):
+    c = wl.make_random(1, 2, 300, 1000, 128, seed=35)
+    check_all_rows(c, what=f"causal, split {n_split}", causal=True,
+                   flags=binding.VIDATTN_SPLIT_KV(n_split))
+
+
+def test_key_splits_more_than_key_tiles():
+    """Two key tiles split five ways: three ranges are empty."""
+    c = wl.make_random(1, 1, 200, 129, 64, seed=36)
+    check_all_rows(c, what="split 5 over 2 tiles", flags=binding.VIDATTN_SPLIT_KV(5))
+
+
+def test_auto_split_long_keys():
+    """A few query blocks over many keys (4 units, 64 key tiles): the
+    heuristic splits the keys 8 ways; the result matches the oracle and the
+    unsplit launch to within bf16 rounding."""
+    c = wl.make_random(1, 2, 512, 8192, 64, seed=37)
+    assert binding.split_count(None, 1, 2, 512, 8192) == 8
+    o1, l1 = run_gpu(c)
+    ro, rl = oracle.attn_fwd(c["q"], c["k"], c["v"], None, None, c["scale"])
+    compare(bf16_to_f64(o1), l1.double().cpu().numpy(), ro, rl, "auto split 8")
+    o2, l2 = run_gpu(c, flags=binding.VIDATTN_SPLIT_KV(1))
+    d = (o1.double() - o2.double()).abs()
+    assert float(d.max()) <= 1e-2 and float((l1 - l2).abs().max()) <= 1e-4
+
+
+# ------------------------------------------------ persistent launches
+# Many short units (more than the 148 SMs, few key tiles each): the launch
+# is persistent, so every CTA carries its barrier phases, Q buffers and
+# tile lists across several units.
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("mode", ["plain", "ids", "causal"])
+def test_persistent_many_short_units(D, mode):
+    B, H, S = 2, 40, 1000       # 2 x 40 x 4 = 320 units of 8 key tiles
+    seg = None
+    if mode == "ids":
+        seg = wl.segment_ids(((700, 0), (200, 1), (100, 2)), B)
+    c = wl.make_random(B, H, S, S, D, 38 + D, seg, None if seg is None else seg.copy())
+    check_all_rows(c, what=f"persistent {mode} D{D}", causal=(mode == "causal"))
 
 
 # ----------------------------------------------------------- segment layouts
@@ -41,9 +107,10 @@ def runs_case(B, H, runs, D, seed):
 
 
 @pytest.mark.parametrize("D", [64, 128])
-def test_video_text_pad_segments(D):
+@pytest.mark.parametrize("n_split", [0, 1])
+def test_video_text_pad_segments(D, n_split):
     c = runs_case(2, 3, ((700, 0), (140, 1), (37, 2)), D, 31)
-    check_all_rows(c, what="video/text/pad")
+    check_all_rows(c, what=f"video/text/pad split {n_split}", flags=binding.VIDATTN_SPLIT_KV(n_split))
 
 
 @pytest.mark.parametrize("D", [64, 128])
@@ -109,16 +176,19 @@ def test_peaked_softmax_with_head_scaling():
     check_all_rows(c, what="peaked")
 
 
+@pytest.mark.parametrize("n_split", [0, 1])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("with_ids", [False, True])
 @pytest.mark.parametrize("pattern", ["per_tile", "within_tile"])
-def test_running_offset_overflow_takes_exact_path(D, with_ids, pattern):
+def test_running_offset_overflow_takes_exact_path(D, with_ids, pattern, n_split):
     """Keys scaled so that scores grow along the sequence: the offset a row
     takes from its first key tile goes stale by far more than 2^32 in P, and
     the kernel must fall back to the exact path (tile max, rescale of O and
     the row sum) and still match the oracle.  per_tile: 128-key tiles scaled
     0.05x .. 16x (the whole tile overflows).  within_tile: 64-key halves
-    scaled so that only the second half of a tile overflows."""
+    scaled so that only the second half of a tile overflows.  n_split 1
+    keeps every key tile of a row in one unit (the launch would split this
+    short call otherwise, 0), so the running offset meets the later tiles."""
     B, H, S_q, S_kv = 1, 2, 300, 640
     rng = np.random.Generator(np.random.PCG64(46 + D))
     q = rng.standard_normal((B, H, S_q, D), dtype=np.float32)
@@ -135,7 +205,8 @@ def test_running_offset_overflow_takes_exact_path(D, with_ids, pattern):
     if with_ids:   # one id everywhere: the listed-tile path, same result
         c["seg_q"] = np.zeros((B, S_q), np.int32)
         c["seg_kv"] = np.zeros((B, S_kv), np.int32)
-    check_all_rows(c, what=f"stale offset {pattern} D{D} ids={with_ids}")
+    check_all_rows(c, what=f"stale offset {pattern} D{D} ids={with_ids} split={n_split}",
+                   flags=binding.VIDATTN_SPLIT_KV(n_split))
 
 
 def test_scale_zero_with_segments_gives_segment_means():
@@ -283,9 +354,11 @@ def test_streams_other_than_the_current_one():
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("S_q,S_kv", [(128, 128), (300, 300), (257, 513), (513, 257),
                                       (1000, 1000), (100, 700)])
-def test_causal_shapes(S_q, S_kv, D):
+@pytest.mark.parametrize("n_split", [0, 1])
+def test_causal_shapes(S_q, S_kv, D, n_split):
     c = wl.make_random(2, 2, S_q, S_kv, D, seed=S_q + 3 * S_kv + D)
-    check_all_rows(c, causal=True, what=f"causal Sq{S_q} Skv{S_kv} D{D}")
+    check_all_rows(c, causal=True, what=f"causal Sq{S_q} Skv{S_kv} D{D} split {n_split}",
+                   flags=binding.VIDATTN_SPLIT_KV(n_split))
 
 
 @pytest.mark.parametrize("D", [64, 128])

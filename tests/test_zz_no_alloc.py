@@ -6,9 +6,10 @@ first use.
 
 The GPU test calls it through the C ABI several times in a row, with
 different shapes and segment layouts, through the same fixed array.  Each
-result must equal the allocating entry point vidattn_fwd's bit for bit (the
-same classifier and attention kernel run on the same summaries, only stored
-elsewhere) and match the fp64 oracle under the parity tolerances.  One case
+result must equal the allocating entry point's unsplit launch bit for bit
+(vidattn_fwd_ex with VIDATTN_SPLIT_KV(1): the same classifier and attention
+kernel run on the same summaries, only stored elsewhere) and match the fp64
+oracle under the parity tolerances.  One case
 has two samples with different ids, so a wrong per-sample offset into the
 array would show.  This file is collected last, so a run that stops at the
 first failure has already run every other test."""
@@ -45,6 +46,11 @@ def _run(fn, c):
     return out, lse
 
 
+def _unsplit(q, k, v, sq, sk, out, lse, B, H, S_q, S_kv, D, scale):
+    return binding.vidattn_fwd_ex(q, k, v, sq, sk, out, lse, B, H, S_q, S_kv, D, scale,
+                                  binding.VIDATTN_SPLIT_KV(1))
+
+
 def _against_oracle(c, out, lse):
     h = c["host"]
     ro, rl = oracle.attn_fwd(h["q"], h["k"], h["v"], h["seg_q"], h["seg_kv"], h["scale"])
@@ -72,7 +78,7 @@ def test_no_alloc_matches_allocating_entry_point_on_calls_in_a_row():
     first = None
     for c in cases + cases[:1]:           # calls in a row through the same array, then again
         out_n, lse_n = _run(binding.vidattn_fwd_noalloc, c)
-        out_r, lse_r = _run(binding.vidattn_fwd, c)
+        out_r, lse_r = _run(_unsplit, c)
         assert torch.equal(out_n.view(torch.int16), out_r.view(torch.int16))
         assert torch.equal(lse_n.view(torch.int32), lse_r.view(torch.int32))
         _against_oracle(c, out_n, lse_n)

@@ -54,8 +54,10 @@ def load_library():
     lib.vidattn_release.restype = None
     lib.vidattn_device_status.argtypes = [p]
     lib.vidattn_device_status.restype = i32
-    lib.vidattn_kernels_per_call.argtypes = [p, p, i32, i32, i32, i32, i32]
+    lib.vidattn_kernels_per_call.argtypes = [p, p, i32, i32, i32, i32, i32, i32]
     lib.vidattn_kernels_per_call.restype = i32
+    lib.vidattn_split_count.argtypes = [p, i32, i32, i32, i32, i32]
+    lib.vidattn_split_count.restype = i32
     lib.vidattn_selftest_timeout.argtypes = [i32, p]
     lib.vidattn_selftest_timeout.restype = i32
     lib.vidattn_fwd_window.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, f32,
@@ -201,9 +203,21 @@ def selftest_timeout(timeout_us: int, stream=None) -> int:
     return load_library().vidattn_selftest_timeout(int(timeout_us), _stream(stream))
 
 
-def kernels_per_call(seg_q, seg_kv, B, H, S_q, S_kv, D) -> int:
+def kernels_per_call(seg_q, seg_kv, B, H, S_q, S_kv, D, flags=0) -> int:
     return load_library().vidattn_kernels_per_call(_ptr(seg_q), _ptr(seg_kv), int(B), int(H),
-                                                   int(S_q), int(S_kv), int(D))
+                                                   int(S_q), int(S_kv), int(D), int(flags))
+
+
+def split_count(seg_q, B, H, S_q, S_kv, flags=0) -> int:
+    """Key splits a vidattn_fwd_ex call with these arguments uses (the
+    library's launch heuristic, or the VIDATTN_SPLIT_KV request in flags)."""
+    return load_library().vidattn_split_count(_ptr(seg_q), int(B), int(H), int(S_q), int(S_kv),
+                                              int(flags))
+
+
+def VIDATTN_SPLIT_KV(n: int) -> int:
+    """vidattn_fwd_ex flag: split every 256-row query block's keys into n ranges."""
+    return (int(n) & 0xFF) << 8
 
 
 def attention(q, k, v, seg_q=None, seg_kv=None, scale=None, stream=None, causal=False):

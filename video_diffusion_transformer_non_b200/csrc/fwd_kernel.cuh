@@ -42,6 +42,7 @@
 // ids or coordinates are staged per warp in shared memory and each row builds
 // a 128-bit mask from them.
 #pragma once
+#include <climits>
 #include <cstdint>
 #include <cuda.h>
 
@@ -60,6 +61,9 @@ constexpr int kErrTimeout = 1;
 // there are at most this many key tiles (S_kv <= 262144); beyond, roles walk
 // the summaries in global memory.
 constexpr int kMaxListedTiles = 2048;
+// Threads that read a unit's tile list (loader warp, MMA warp, softmax
+// warpgroups); each arrives once when it is done with the list.
+constexpr int kListReaders = 320;
 
 struct FwdParams {
   const int32_t* seg_q;     // [B,S_q] or null
@@ -78,6 +82,13 @@ struct FwdParams {
   int* err;                 // device error word (bit kErrTimeout: a wait timed out)
   int H, S_q, S_kv;
   int n_q_tiles, n_kv_tiles;
+  int n_pairs;              // 256-row query blocks per (b, h): ceil(S_q / 256)
+  int n_split;              // key splits per query block (1: no split)
+  int n_units;              // B * H * n_pairs * n_split work units
+  // n_split > 1: per split, O / l and the log-sum-exp of each row, fp32
+  // [B*H][n_split][S_q][D] and [B*H][n_split][S_q], merged by split_combine_kernel
+  float* part_o;
+  float* part_lse;
   int causal;               // nonzero: key j visible to query i only if j <= i + causal_off
   int causal_off;           // S_kv - S_q (the last query aligned with the last key)
   float c;                  // scale * log2(e)
@@ -109,15 +120,17 @@ struct FwdCfg {
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   // q_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] drain[1] s_free[2]
-  static constexpr int kNumBars = 2 + 2 * kStages + 9;
-  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;   // tmem addr, abort flag
-  static constexpr int kOffWarpCnt = kOffMisc + 16;         // 12 ints (list building)
-  static constexpr int kOffList = kOffWarpCnt + 64;         // active key tiles
+  // q_empty[1] list_full[2] list_empty[2]
+  static constexpr int kNumBars = 2 + 2 * kStages + 14;
+  // tmem addr, abort flag, the two lists' lengths
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+  static constexpr int kOffList = kOffMisc + 16;            // two lists of key tiles
   // per softmax warp: the ids or window coordinates of the 128 keys of the
   // masked key tile it is working on (read as int4: 16-byte aligned)
-  static constexpr int kOffKinfo = (kOffList + 4 * kMaxListedTiles + 127) & ~127;
+  static constexpr int kOffKinfo = (kOffList + 2 * 4 * kMaxListedTiles + 127) & ~127;
   static_assert(kOffKinfo % 16 == 0, "int4 reads of the key-info slots");
   static constexpr int kSmemBytes = kOffKinfo + 8 * kBN * 4 + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 227 * 1024, "one CTA's shared memory on sm_100");
   // P in its own tensor-memory columns (D = 64, where they fit) instead of
   // over the first half of S: the next Q K^T of a tile need not wait for
   // the P V that reads its P.
@@ -460,21 +473,6 @@ __device__ __forceinline__ KvWalk make_walk(const FwdParams& p, int b, int pair,
   return walk;
 }
 
-// The sequence of key tiles a CTA visits, as every role walks it.
-//   listed: entry t of a shared-memory list: bits 0-29 = j, bit 30 + i =
-//           "Q tile i needs the masked path on this key tile";
-//   otherwise: the global walk (with ids) or every tile (without).
-struct KvSched {
-  const int* list;
-  int n_list;
-  KvWalk walk;
-  // j of the t-th visited tile (prev_j: the (t-1)-th, -1 for t = 0); n_kv when done.
-  __device__ __forceinline__ int tile(int t, int prev_j) const {
-    if (list != nullptr) return t < n_list ? (list[t] & 0x3FFFFFFF) : walk.n_kv;
-    return walk.next(prev_j + 1);
-  }
-};
-
 template <int D>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t sQ, uint32_t sK) {
   using C = FwdCfg<D>;
@@ -501,12 +499,80 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   }
 }
 
+// One work unit of the persistent kernel: (b, h, 256-row query block `pair`,
+// key split `split` of n_split).
+struct Unit {
+  int b, h, pair, split;
+};
+// Units are numbered split fastest, then query block, then head: one head's
+// units run close together in time (its K and V stay in L2).  With the
+// causal limit the query blocks of a head go longest first (the last block
+// sees the most keys), so no long unit trails at the end of the launch.
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
+  Unit x;
+  x.split = u % p.n_split;
+  const int r = u / p.n_split;
+  const int pp = r % p.n_pairs;
+  const int bh = r / p.n_pairs;
+  x.b = bh / p.H;
+  x.h = bh - x.b * p.H;
+  x.pair = p.causal ? p.n_pairs - 1 - pp : pp;
+  return x;
+}
+
+// The key tiles a unit visits: positions [t0, t1) of the pair's visit
+// sequence (its listed tiles, or every tile below the causal end, or the
+// global walk with ids beyond the list's capacity, where n_split is 1).
+struct UnitSched {
+  const int* list;   // the unit's listed tiles, or null
+  int t0, t1;
+  int n_kv;          // one past the last key tile any row of the pair can see
+  KvWalk walk;
+  // j of position t (prev_j: j of position t - 1, or t0 - 1 at the start);
+  // n_kv once the unit's range is done
+  __device__ __forceinline__ int tile(int t, int prev_j) const {
+    if (t >= t1) return n_kv;
+    if (list != nullptr) return list[t] & 0x3FFFFFFF;
+    return walk.next(prev_j + 1);
+  }
+};
+
+__device__ __forceinline__ UnitSched unit_sched(const FwdParams& p, const Unit& x,
+                                                const int* list, int n_list) {
+  UnitSched s;
+  s.list = list;
+  s.walk = make_walk(p, x.b, x.pair);
+  s.n_kv = s.walk.n_kv;
+  // positions of the whole pair: listed tiles, the global walk (ids beyond
+  // the list's capacity: its length is not known up front; n_split is 1) or
+  // every tile below the causal end
+  const int total = list != nullptr ? n_list : (s.walk.kv_sum != nullptr ? INT_MAX : s.n_kv);
+  if (p.n_split == 1) {
+    s.t0 = 0;
+    s.t1 = total;
+  } else {
+    s.t0 = int((int64_t(total) * x.split) / p.n_split);
+    s.t1 = int((int64_t(total) * (x.split + 1)) / p.n_split);
+  }
+  return s;
+}
+
 // kEmu: exponentials per 16 keys computed on the FMA pipe instead of MUFU.
 // kMaskFast: masked key tiles (D = 128) take the running-offset path with
 // their hidden keys' scores set to -inf, instead of the two-pass exact path
 // (the variant for 3D neighbourhood windows, where nearly every visited tile
 // is masked; elsewhere the extra code costs the unmasked tiles registers).
-template <int D, int kEmu, bool kMaskFast>
+//
+// kSplit: the launch splits the keys (FwdParams::n_split > 1); the epilogue
+// writes each split's partial result for split_combine_kernel instead of out
+// and lse.
+// kPersist: the grid holds at most one CTA per SM, and CTA i works on units
+// i, i + gridDim.x, ...  Every barrier phase runs on across units, so the
+// loader fetches the next unit's Q and first K/V tiles and the MMA warp
+// issues its first Q K^T while the softmax warps still write the previous
+// unit's output.  Otherwise one CTA per unit, scheduled by the hardware as
+// SMs free up.
+template <int D, int kEmu, bool kMaskFast, bool kPersist, bool kSplit>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     vidattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -523,14 +589,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int b = blockIdx.z;
-  const int h = blockIdx.y;
-  const int bh = b * p.H + h;
-  // 256-row query block of this CTA.  With the causal limit, later blocks see
-  // more keys: they are handed out first (the hardware starts CTAs in index
-  // order), so the longest work does not trail at the end of the launch.
-  const int pair = p.causal ? int(gridDim.x) - 1 - int(blockIdx.x) : int(blockIdx.x);
-  const int m0 = pair * 2 * kBM;
+  // the units of this CTA: every gridDim.x-th from blockIdx.x when
+  // persistent; else the grid holds one CTA per unit and the loops below run
+  // once (a trip count the compiler sees, so nothing carries across units)
+  const int u_end = kPersist ? p.n_units : int(blockIdx.x) + 1;
+  const int u_step = kPersist ? int(gridDim.x) : 1;
 
   const uint32_t sQ[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
   auto sKV = [&](int s) { return sbase + C::kOffKV + s * C::kTileBytes; };
@@ -543,8 +606,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   auto o_full = [&](int i) { return bar(6 + 2 * C::kStages + i); };
   const uint32_t drain_bar = bar(8 + 2 * C::kStages);
   auto s_free = [&](int i) { return bar(9 + 2 * C::kStages + i); };
+  // the Q tiles may be overwritten (every Q K^T of the unit has run)
+  const uint32_t q_empty = bar(11 + 2 * C::kStages);
+  // tile lists, double-buffered: written (list_full) / read by every role (list_empty)
+  auto list_full = [&](int i) { return bar(12 + 2 * C::kStages + i); };
+  auto list_empty = [&](int i) { return bar(14 + 2 * C::kStages + i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  int* list_count = reinterpret_cast<int*>(smem + C::kOffMisc + 8);   // [2]
+  int* list_base = reinterpret_cast<int*>(smem + C::kOffList);          // [2][kMaxListedTiles]
 
   if (threadIdx.x == 0) {
     mbar_init(q_full(0), 1);
@@ -558,8 +628,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(p_full(i), 128);
       mbar_init(o_full(i), 1);
       mbar_init(s_free(i), 128);
+      mbar_init(list_full(i), 32);
+      mbar_init(list_empty(i), kListReaders);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(q_empty, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -572,594 +645,710 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-
   const bool has_sum = p.q_sum != nullptr;      // tile summaries: ids or window boxes
   const bool has_win = p.coord_q != nullptr;
   const bool has_seg = has_sum && !has_win;
-  // key tiles visited end here (causal: past the last key any row sees)
-  const int n_kv = causal_end(p, pair);
+  // With summaries, warp 10 lists each unit's visited key tiles (id ranges or
+  // window boxes that meet its queries') with per-Q-tile mask bits, so no
+  // role touches global memory to find its next tile; beyond the list's
+  // capacity the roles walk the summaries in global memory.
+  const bool listed = has_sum && p.n_kv_tiles <= kMaxListedTiles;
 #ifdef VIDATTN_TRACE
-  const bool trace_cta = p.trace != nullptr && blockIdx.x == gridDim.x / 2 &&
-                         blockIdx.y == gridDim.y / 2 && blockIdx.z == 0;
+  const bool trace_cta = p.trace != nullptr && blockIdx.x == gridDim.x / 2;
 #endif
-
-  // With ids: compact this CTA's visited key tiles (id ranges that meet its
-  // queries' range) into shared memory, with per-Q-tile mask bits, so no role
-  // touches global memory to find its next tile.
-  int* tile_list = reinterpret_cast<int*>(smem + C::kOffList);
-  int n_list = 0;
-  const bool listed = has_sum && n_kv <= kMaxListedTiles;
-  if (listed) {
-    int4 q0, q1;
-    const KvWalk w = make_walk(p, b, pair, 0, &q0);
-    make_walk(p, b, pair, 1, &q1);
-    const bool ragged = (p.S_kv % kBN) != 0;
-    int* warp_cnt = reinterpret_cast<int*>(smem + C::kOffWarpCnt);
-    for (int c0 = 0; c0 < n_kv; c0 += kFwdThreads) {
-      const int jj = c0 + threadIdx.x;
-      bool act = false;
-      int entry = 0;
-      if (jj < n_kv) {
-        const int4 ks = __ldg(p.kv_sum + static_cast<int64_t>(b) * p.n_kv_tiles + jj);
-        const bool last_ragged = ragged && jj == p.n_kv_tiles - 1;
-        bool m0, m1;
-        if (has_win) {
-          act = win_tile_meets(p, q0, q1, ks);
-          m0 = last_ragged || !win_tile_full(p, q0, ks);
-          m1 = last_ragged || !win_tile_full(p, q1, ks);
-        } else {
-          act = !(ks.y < w.qmin || ks.x > w.qmax);
-          m0 = last_ragged || !(q0.z && ks.z && q0.x == ks.x) || causal_partial(p, pair, 0, jj);
-          m1 = last_ragged || !(q1.z && ks.z && q1.x == ks.x) || causal_partial(p, pair, 1, jj);
-        }
-        entry = jj | (m0 ? (1 << 30) : 0) | (m1 ? int(1u << 31) : 0);
-      }
-      const unsigned ballot = __ballot_sync(0xffffffffu, act);
-      if (lane == 0) warp_cnt[warp] = __popc(ballot);
-      __syncthreads();
-      int off = n_list, total = 0;
-#pragma unroll
-      for (int w2 = 0; w2 < kFwdThreads / 32; ++w2) {
-        const int cnt = warp_cnt[w2];
-        off += (w2 < warp) ? cnt : 0;
-        total += cnt;
-      }
-      if (act) tile_list[off + __popc(ballot & ((1u << lane) - 1u))] = entry;
-      n_list += total;
-      __syncthreads();
-    }
-  }
+  // list of the k-th unit of this CTA, once warp 10 has written it
+  auto wait_list = [&](int k, const int** list, int* n_list) -> bool {
+    *list = nullptr;
+    *n_list = 0;
+    if (!listed) return true;
+    const int buf = k & 1;
+    if (!warp_wait_phase(list_full(buf), uint32_t(k >> 1) & 1u, abort_flag, p.err)) return false;
+    *list = list_base + buf * kMaxListedTiles;
+    *n_list = *reinterpret_cast<volatile int*>(list_count + buf);
+    return true;
+  };
+  auto release_list = [&](int k) {
+    if (listed) mbar_arrive(list_empty(k & 1));
+  };
 
   // Register split: the launch gives 168 per thread (384 x 168 = 64512);
-  // warpgroup 2 (MMA, TMA, idle warps) drops so the two softmax warpgroups
-  // can rise: D = 128: 128 x 96 + 256 x 200 = 63488; D = 64 (whose softmax
-  // keeps its S row in registers): 128 x 64 + 256 x 216 = 63488; both
-  // <= 64512.  Each warpgroup executes its setmaxnreg at the head of its
-  // own branch.
+  // warpgroup 2 (MMA, TMA, list builder, idle warp) drops so the two softmax
+  // warpgroups can rise.  Per variant, a split without register spills
+  // (ptxas, for the default kEmu of each head dim): D = 128: 128 x 128 +
+  // 256 x 184 = 63488; D = 64 persistent: 128 x 96 + 256 x 200 = 63488; the
+  // others (D = 64, the window variant, whose softmax also holds the mask):
+  // 128 x 104 + 256 x 192 = 62464; all <= 64512.  Each warpgroup executes
+  // its setmaxnreg at the head of its own branch.
   if (warp >= 8) {
-  if constexpr (D == 128) {
+  if constexpr (D == 128 && !kMaskFast) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 128;" ::: "memory");
+  } else if constexpr (kPersist) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
   } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;" ::: "memory");
   }
   if (warp == 9) {
     // ------------------------------------------------------------ TMA loads
-    {  // the whole warp runs the loop; one elected lane issues
-      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, pair)};
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-      }
-      int t = 0;
-      int j = sched.tile(0, -1);
-      int n = 0;   // K/V loads issued
-      bool ok = true;
-      if (j < n_kv) {
+    // the whole warp runs the loop; one elected lane issues
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    int n = 0;    // K/V loads issued (ring position), over all units
+    int kq = 0;   // units with at least one tile so far (Q loads)
+    bool ok = true;
+    for (int u = blockIdx.x, k = 0; ok && u < u_end; u += u_step, ++k) {
+      const int* list;
+      int n_list;
+      ok = wait_list(k, &list, &n_list);
+      if (!ok) break;
+      const Unit x = decode_unit(p, u);
+      const UnitSched sched = unit_sched(p, x, list, n_list);
+      const int bh = x.b * p.H + x.h;
+      const int m0 = x.pair * 2 * kBM;
+      int t = sched.t0;
+      int j = sched.tile(t, t - 1);
+      if (j < sched.n_kv) {
+        if (kq > 0) ok = warp_wait_phase(q_empty, uint32_t(kq - 1) & 1u, abort_flag, p.err);
+        if (!ok) break;
         mbar_arrive_expect_tx_elect(q_full(0), C::kTileBytes);
         for (int s = 0; s < C::kSub; ++s)
           tma_load_3d_elect(sQ[0] + s * C::kSubBytes, &tm_q, q_full(0), s * 64, m0, bh);
-      }
-      bool first = true;
-      while (ok && j < n_kv) {
-        for (int which = 0; which < 2 && ok; ++which) {   // K_j then V_j
-          const int st = n % C::kStages;
-          VIDATTN_TR(3, n, 0);
-          ok = warp_wait_phase(kv_empty(st), ((n / C::kStages) & 1) ^ 1, abort_flag, p.err);
-          VIDATTN_TR(3, n, 1);
-          if (!ok) break;
-          mbar_arrive_expect_tx_elect(kv_full(st), C::kTileBytes);
-          for (int s = 0; s < C::kSub; ++s)
-            tma_load_3d_elect(sKV(st) + s * C::kSubBytes, which ? &tm_v : &tm_k, kv_full(st), s * 64,
-                        j * kBN, bh);
-          ++n;
-          if (first) {
-            first = false;
-            mbar_arrive_expect_tx_elect(q_full(1), C::kTileBytes);
+        bool first = true;
+        while (ok && j < sched.n_kv) {
+          for (int which = 0; which < 2 && ok; ++which) {   // K_j then V_j
+            const int st = n % C::kStages;
+            VIDATTN_TR(3, n, 0);
+            ok = warp_wait_phase(kv_empty(st), ((n / C::kStages) & 1) ^ 1, abort_flag, p.err);
+            VIDATTN_TR(3, n, 1);
+            if (!ok) break;
+            mbar_arrive_expect_tx_elect(kv_full(st), C::kTileBytes);
             for (int s = 0; s < C::kSub; ++s)
-              tma_load_3d_elect(sQ[1] + s * C::kSubBytes, &tm_q, q_full(1), s * 64, m0 + kBM, bh);
+              tma_load_3d_elect(sKV(st) + s * C::kSubBytes, which ? &tm_v : &tm_k, kv_full(st),
+                                s * 64, j * kBN, bh);
+            ++n;
+            if (first) {
+              first = false;
+              mbar_arrive_expect_tx_elect(q_full(1), C::kTileBytes);
+              for (int s = 0; s < C::kSub; ++s)
+                tma_load_3d_elect(sQ[1] + s * C::kSubBytes, &tm_q, q_full(1), s * 64, m0 + kBM,
+                                  bh);
+            }
           }
+          j = sched.tile(++t, j);
         }
-        j = sched.tile(++t, j);
+        ++kq;
       }
-      if (!ok) {
-        // Let the loads already in flight land before the CTA can exit.
-        for (int k = (n > C::kStages ? n - C::kStages : 0); k < n; ++k) {
-          const int st = k % C::kStages;
-          volatile int never = 0;
-          warp_wait_phase(kv_full(st), (k / C::kStages) & 1, &never, p.err);
-        }
+      __syncwarp();
+      release_list(k);
+    }
+    if (!ok) {
+      // Let the loads already in flight land before the CTA can exit.
+      for (int k = (n > C::kStages ? n - C::kStages : 0); k < n; ++k) {
+        const int st = k % C::kStages;
+        volatile int never = 0;
+        warp_wait_phase(kv_full(st), (k / C::kStages) & 1, &never, p.err);
       }
     }
     __syncwarp();
   } else if (warp == 8) {
     // ------------------------------------------------------- tensor core
-    if (C::kSepP) {  // the whole warp runs the loop; one elected lane issues
-      // Order per tile t: S0 = Q0 K_{t+1}^T once S0_t is read, O0 += P0 V_t,
-      // S1 = Q1 K_{t+1}^T once S1_t is read, O1 += P1 V_t.  K_t is load 2t
-      // and V_t load 2t+1 of the ring.
-      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, pair)};
-      int j = sched.tile(0, -1);
-      if (j < n_kv) {
-        auto stage = [&](int idx) { return idx % C::kStages; };
-        auto par = [&](int idx) { return uint32_t(idx / C::kStages) & 1u; };
-        int t = 0;
-        bool ok = warp_wait_phase(q_full(0), 0, abort_flag, p.err);
-        ok = ok && warp_wait_phase(kv_full(stage(0)), par(0), abort_flag, p.err);
-        if (ok) {
-          tc_fence_after();
-          issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(stage(0)));
-          mma_commit_elect(s_full(0));
-          ok = warp_wait_phase(q_full(1), 0, abort_flag, p.err);
-        }
-        if (ok) {
-          tc_fence_after();
-          issue_qk<D>(tmem + C::kTmemS + 128, sQ[1], sKV(stage(0)));
-          mma_commit_elect(s_full(1));
-          mma_commit_elect(kv_empty(stage(0)));
-        }
-        while (ok) {
-          const int jn = sched.tile(t + 1, j);
-          const bool more = jn < n_kv;
-          const int kn = 2 * (t + 1), vi = 2 * t + 1;
-          VIDATTN_TR(0, t, 0);
-          // both tiles' data first (see the aliased loop)
-          ok = warp_wait_phase(kv_full(stage(vi)), par(vi), abort_flag, p.err);
-          if (ok && more) ok = warp_wait_phase(kv_full(stage(kn)), par(kn), abort_flag, p.err);
-          if (!ok) break;
-          if (more) {
-            ok = warp_wait_phase(s_free(0), t & 1, abort_flag, p.err);
-            VIDATTN_TR(0, t, 1);
-            if (!ok) break;
+    // the whole warp runs the loop; one elected lane issues
+    auto stage = [&](int idx) { return idx % C::kStages; };
+    auto par = [&](int idx) { return uint32_t(idx / C::kStages) & 1u; };
+    int n = 0;    // K/V tiles consumed (ring position), over all units
+    int T = 0;    // key tiles done by this CTA, over all units (barrier parities)
+    int kq = 0;   // units with at least one tile so far
+    bool ok = true;
+    for (int u = blockIdx.x, k = 0; ok && u < u_end; u += u_step, ++k) {
+      const int* list;
+      int n_list;
+      ok = wait_list(k, &list, &n_list);
+      if (!ok) break;
+      const Unit x = decode_unit(p, u);
+      const UnitSched sched = unit_sched(p, x, list, n_list);
+      int t = sched.t0;
+      int j = sched.tile(t, t - 1);
+      if (j < sched.n_kv) {
+        const uint32_t qpar = uint32_t(kq) & 1u;
+        if (C::kSepP) {
+          // Order per tile t: S0 = Q0 K_{t+1}^T once S0_t is read, O0 += P0 V_t,
+          // S1 = Q1 K_{t+1}^T once S1_t is read, O1 += P1 V_t.  K_t is load 2t
+          // and V_t load 2t+1 of the ring.
+          ok = warp_wait_phase(q_full(0), qpar, abort_flag, p.err);
+          ok = ok && warp_wait_phase(kv_full(stage(n)), par(n), abort_flag, p.err);
+          // S0 of the previous unit's last tile has been read
+          ok = ok && (T == 0 || warp_wait_phase(s_free(0), uint32_t(T - 1) & 1u, abort_flag, p.err));
+          const int k0 = n++;
+          if (ok) {
             tc_fence_after();
-            issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(stage(kn)));
+            issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(stage(k0)));
             mma_commit_elect(s_full(0));
-            VIDATTN_TR(0, t, 2);
+            ok = warp_wait_phase(q_full(1), qpar, abort_flag, p.err);
+            ok = ok && (T == 0 || warp_wait_phase(s_free(1), uint32_t(T - 1) & 1u, abort_flag, p.err));
           }
-          ok = warp_wait_phase(p_full(0), t & 1, abort_flag, p.err);
-          VIDATTN_TR(0, t, 3);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv<D>(tmem + C::kTmemO, tmem + C::kTmemP, sKV(stage(vi)), t > 0);
-          mma_commit_elect(o_full(0));
-          VIDATTN_TR(0, t, 4);
-          if (more) {
-            ok = warp_wait_phase(s_free(1), t & 1, abort_flag, p.err);
-            VIDATTN_TR(0, t, 5);
+          if (ok) {
+            tc_fence_after();
+            issue_qk<D>(tmem + C::kTmemS + 128, sQ[1], sKV(stage(k0)));
+            mma_commit_elect(s_full(1));
+            mma_commit_elect(kv_empty(stage(k0)));
+          }
+          bool first = true;
+          while (ok) {
+            const int jn = sched.tile(t + 1, j);
+            const bool more = jn < sched.n_kv;
+            if (!more) mma_commit_elect(q_empty);   // the unit's last Q K^T is issued
+            const int vi = n++;
+            VIDATTN_TR(0, T, 0);
+            // both tiles' data first (see the aliased loop)
+            ok = warp_wait_phase(kv_full(stage(vi)), par(vi), abort_flag, p.err);
+            int kn = 0;
+            if (ok && more) {
+              kn = n++;
+              ok = warp_wait_phase(kv_full(stage(kn)), par(kn), abort_flag, p.err);
+            }
+            if (!ok) break;
+            if (more) {
+              ok = warp_wait_phase(s_free(0), uint32_t(T) & 1u, abort_flag, p.err);
+              VIDATTN_TR(0, T, 1);
+              if (!ok) break;
+              tc_fence_after();
+              issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(stage(kn)));
+              mma_commit_elect(s_full(0));
+              VIDATTN_TR(0, T, 2);
+            }
+            ok = warp_wait_phase(p_full(0), uint32_t(T) & 1u, abort_flag, p.err);
+            VIDATTN_TR(0, T, 3);
             if (!ok) break;
             tc_fence_after();
-            issue_qk<D>(tmem + C::kTmemS + 128, sQ[1], sKV(stage(kn)));
-            mma_commit_elect(s_full(1));
-            mma_commit_elect(kv_empty(stage(kn)));
-            VIDATTN_TR(0, t, 6);
+            issue_pv<D>(tmem + C::kTmemO, tmem + C::kTmemP, sKV(stage(vi)), !first);
+            mma_commit_elect(o_full(0));
+            VIDATTN_TR(0, T, 4);
+            if (more) {
+              ok = warp_wait_phase(s_free(1), uint32_t(T) & 1u, abort_flag, p.err);
+              VIDATTN_TR(0, T, 5);
+              if (!ok) break;
+              tc_fence_after();
+              issue_qk<D>(tmem + C::kTmemS + 128, sQ[1], sKV(stage(kn)));
+              mma_commit_elect(s_full(1));
+              mma_commit_elect(kv_empty(stage(kn)));
+              VIDATTN_TR(0, T, 6);
+            }
+            ok = warp_wait_phase(p_full(1), uint32_t(T) & 1u, abort_flag, p.err);
+            VIDATTN_TR(0, T, 7);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv<D>(tmem + C::kTmemO + D, tmem + C::kTmemP + C::kPStride, sKV(stage(vi)),
+                        !first);
+            mma_commit_elect(o_full(1));
+            mma_commit_elect(kv_empty(stage(vi)));
+            VIDATTN_TR(0, T, 8);
+            ++T;
+            first = false;
+            if (!more) break;
+            j = jn;
+            ++t;
           }
-          ok = warp_wait_phase(p_full(1), t & 1, abort_flag, p.err);
-          VIDATTN_TR(0, t, 7);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv<D>(tmem + C::kTmemO + D, tmem + C::kTmemP + C::kPStride, sKV(stage(vi)),
-                      t > 0);
-          mma_commit_elect(o_full(1));
-          mma_commit_elect(kv_empty(stage(vi)));
-          VIDATTN_TR(0, t, 8);
-          if (!more) break;
-          j = jn;
-          ++t;
-        }
-        mma_commit_elect(drain_bar);
-        volatile int never = 0;
-        warp_wait_phase(drain_bar, 0, &never, p.err);
-      }
-    } else {
-      const KvSched sched{listed ? tile_list : nullptr, n_list, make_walk(p, b, pair)};
-      int j = sched.tile(0, -1);
-      if (j < n_kv) {
-        int n = 0;   // K/V tiles consumed
-        int t = 0;
-        bool ok = warp_wait_phase(q_full(0), 0, abort_flag, p.err);
-        int ks = n % C::kStages;
-        ok = ok && warp_wait_phase(kv_full(ks), (n / C::kStages) & 1, abort_flag, p.err);
-        ++n;
-        if (ok) {
-          tc_fence_after();
-          issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(ks));
-          mma_commit_elect(s_full(0));
-          ok = warp_wait_phase(q_full(1), 0, abort_flag, p.err);
-        }
-        if (ok) {
-          tc_fence_after();
-          issue_qk<D>(tmem + (C::kTmemS + 128), sQ[1], sKV(ks));
-          mma_commit_elect(s_full(1));
-          mma_commit_elect(kv_empty(ks));
-        }
-        while (ok) {
-          const int vs = n % C::kStages;
-          VIDATTN_TR(0, t, 0);
-          ok = warp_wait_phase(kv_full(vs), (n / C::kStages) & 1, abort_flag, p.err);
+        } else {
+          ok = warp_wait_phase(q_full(0), qpar, abort_flag, p.err);
+          const int ks = stage(n);
+          ok = ok && warp_wait_phase(kv_full(ks), par(n), abort_flag, p.err);
           ++n;
-          if (!ok) break;
-          const int jn = sched.tile(t + 1, j);
-          // Check that K_{t+1} has landed now, while this warp waits anyway,
-          // instead of between dependent MMAs (an mbarrier read is slow while
-          // a shared-memory-bound Q K^T runs).
-          int ks2 = 0;
-          if (jn < n_kv) {
-            ks2 = n % C::kStages;
-            ok = warp_wait_phase(kv_full(ks2), (n / C::kStages) & 1, abort_flag, p.err);
+          if (ok) {
+            tc_fence_after();
+            issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(ks));
+            mma_commit_elect(s_full(0));
+            ok = warp_wait_phase(q_full(1), qpar, abort_flag, p.err);
+          }
+          if (ok) {
+            tc_fence_after();
+            issue_qk<D>(tmem + (C::kTmemS + 128), sQ[1], sKV(ks));
+            mma_commit_elect(s_full(1));
+            mma_commit_elect(kv_empty(ks));
+          }
+          bool first = true;
+          while (ok) {
+            const int jn = sched.tile(t + 1, j);
+            const bool more = jn < sched.n_kv;
+            if (!more) mma_commit_elect(q_empty);   // the unit's last Q K^T is issued
+            const int vs = stage(n);
+            VIDATTN_TR(0, T, 0);
+            ok = warp_wait_phase(kv_full(vs), par(n), abort_flag, p.err);
             ++n;
             if (!ok) break;
-          }
-          ok = warp_wait_phase(p_full(0), t & 1, abort_flag, p.err);
-          VIDATTN_TR(0, t, 3);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv<D>(tmem + C::kTmemO, tmem + C::kTmemS, sKV(vs), t > 0);
-          mma_commit_elect(o_full(0));
-          VIDATTN_TR(0, t, 4);
-          if (jn < n_kv) {
+            // Check that K_{t+1} has landed now, while this warp waits anyway,
+            // instead of between dependent MMAs (an mbarrier read is slow while
+            // a shared-memory-bound Q K^T runs).
+            int ks2 = 0;
+            if (more) {
+              ks2 = stage(n);
+              ok = warp_wait_phase(kv_full(ks2), par(n), abort_flag, p.err);
+              ++n;
+              if (!ok) break;
+            }
+            ok = warp_wait_phase(p_full(0), uint32_t(T) & 1u, abort_flag, p.err);
+            VIDATTN_TR(0, T, 3);
+            if (!ok) break;
             tc_fence_after();
-            issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(ks2));
-            mma_commit_elect(s_full(0));
-            VIDATTN_TR(0, t, 2);
+            issue_pv<D>(tmem + C::kTmemO, tmem + C::kTmemS, sKV(vs), !first);
+            mma_commit_elect(o_full(0));
+            VIDATTN_TR(0, T, 4);
+            if (more) {
+              tc_fence_after();
+              issue_qk<D>(tmem + C::kTmemS, sQ[0], sKV(ks2));
+              mma_commit_elect(s_full(0));
+              VIDATTN_TR(0, T, 2);
+            }
+            ok = warp_wait_phase(p_full(1), uint32_t(T) & 1u, abort_flag, p.err);
+            VIDATTN_TR(0, T, 7);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv<D>(tmem + (C::kTmemO + D), tmem + (C::kTmemS + 128), sKV(vs), !first);
+            mma_commit_elect(o_full(1));
+            mma_commit_elect(kv_empty(vs));
+            ++T;
+            first = false;
+            if (!more) break;
+            issue_qk<D>(tmem + (C::kTmemS + 128), sQ[1], sKV(ks2));
+            mma_commit_elect(s_full(1));
+            mma_commit_elect(kv_empty(ks2));
+            VIDATTN_TR(0, T, 8);
+            j = jn;
+            ++t;
           }
-          ok = warp_wait_phase(p_full(1), t & 1, abort_flag, p.err);
-          VIDATTN_TR(0, t, 7);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv<D>(tmem + (C::kTmemO + D), tmem + (C::kTmemS + 128), sKV(vs), t > 0);
-          mma_commit_elect(o_full(1));
-          mma_commit_elect(kv_empty(vs));
-          if (jn >= n_kv) break;
-          issue_qk<D>(tmem + (C::kTmemS + 128), sQ[1], sKV(ks2));
-          mma_commit_elect(s_full(1));
-          mma_commit_elect(kv_empty(ks2));
-          VIDATTN_TR(0, t, 8);
-          j = jn;
-          ++t;
         }
-        // Every MMA issued above has finished before TMEM is released.
-        mma_commit_elect(drain_bar);
-        volatile int never = 0;
-        warp_wait_phase(drain_bar, 0, &never, p.err);
+        ++kq;
       }
+      __syncwarp();
+      release_list(k);
+    }
+    // Every MMA issued above has finished before TMEM is released.
+    mma_commit_elect(drain_bar);
+    volatile int never = 0;
+    warp_wait_phase(drain_bar, 0, &never, p.err);
+    __syncwarp();
+  } else if (warp == 10 && listed) {
+    // ------------------------------------------------------- tile lists
+    // For each unit of this CTA: the key tiles the pair visits (id ranges or
+    // window boxes that meet its queries'; with the causal limit, below its
+    // end), entry = j | bit 30 + i when Q tile i needs the mask on tile j.
+    bool ok = true;
+    const bool ragged = (p.S_kv % kBN) != 0;
+    for (int u = blockIdx.x, k = 0; u < u_end; u += u_step, ++k) {
+      const int buf = k & 1;
+      if (k >= 2) ok = warp_wait_phase(list_empty(buf), uint32_t((k >> 1) - 1) & 1u, abort_flag, p.err);
+      if (!ok) break;
+      const Unit x = decode_unit(p, u);
+      int4 q0, q1;
+      const KvWalk w = make_walk(p, x.b, x.pair, 0, &q0);
+      make_walk(p, x.b, x.pair, 1, &q1);
+      const int n_kv = w.n_kv;
+      const int4* kv_sum_b = p.kv_sum + static_cast<int64_t>(x.b) * p.n_kv_tiles;
+      int* list = list_base + buf * kMaxListedTiles;
+      int cnt = 0;
+      for (int c0 = 0; c0 < n_kv; c0 += 32) {
+        const int jj = c0 + lane;
+        bool act = false;
+        int entry = 0;
+        if (jj < n_kv) {
+          const int4 ks = __ldg(kv_sum_b + jj);
+          const bool last_ragged = ragged && jj == p.n_kv_tiles - 1;
+          bool m0, m1;
+          if (has_win) {
+            act = win_tile_meets(p, q0, q1, ks);
+            m0 = last_ragged || !win_tile_full(p, q0, ks);
+            m1 = last_ragged || !win_tile_full(p, q1, ks);
+          } else {
+            act = !(ks.y < w.qmin || ks.x > w.qmax);
+            m0 = last_ragged || !(q0.z && ks.z && q0.x == ks.x) || causal_partial(p, x.pair, 0, jj);
+            m1 = last_ragged || !(q1.z && ks.z && q1.x == ks.x) || causal_partial(p, x.pair, 1, jj);
+          }
+          entry = jj | (m0 ? (1 << 30) : 0) | (m1 ? int(1u << 31) : 0);
+        }
+        const unsigned ballot = __ballot_sync(0xffffffffu, act);
+        if (act) list[cnt + __popc(ballot & ((1u << lane) - 1u))] = entry;
+        cnt += __popc(ballot);
+      }
+      if (lane == 0) list_count[buf] = cnt;
+      __syncwarp();
+      mbar_arrive(list_full(buf));
     }
     __syncwarp();
   }
   } else {
-    if constexpr (D == 128) {
+    if constexpr (D == 128 && !kMaskFast) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
+    } else if constexpr (kPersist) {
       asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
     } else {
-      asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory");
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 192;" ::: "memory");
     }
     // ------------------------------------------------------------ softmax
     const int qi = warp >> 2;                       // which Q tile
     const int r = ((warp & 3) << 5) + lane;         // row in the tile = TMEM lane
-    const int row = m0 + qi * kBM + r;
-    const bool row_valid = row < p.S_q;
-    const int32_t* seg_kv_b = has_seg ? p.seg_kv + static_cast<int64_t>(b) * p.S_kv : nullptr;
-    const int my_seg = (has_seg && row_valid) ? __ldg(p.seg_q + static_cast<int64_t>(b) * p.S_q + row) : 0;
-    const int32_t* coord_kv_b = has_win ? p.coord_kv + static_cast<int64_t>(b) * p.S_kv : nullptr;
-    const int32_t* coord_q_b = has_win ? p.coord_q + static_cast<int64_t>(b) * p.S_q : nullptr;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kTmemS + 128u * qi;
     const uint32_t tO = tmem + lane_off + C::kTmemO + uint32_t(D) * qi;
     const uint32_t tP = tmem + lane_off + C::kTmemP + C::kPStride * qi;
-    int4 my_qs;
-    const KvSched sched{listed ? tile_list : nullptr, n_list,
-                        make_walk(p, b, pair, qi, &my_qs)};
     const float c = p.c;
     const bool ragged_kv = (p.S_kv % kBN) != 0;
     // masked key tiles: their keys' ids or coordinates, staged per warp
     int32_t* kinfo = reinterpret_cast<int32_t*>(smem + C::kOffKinfo) + warp * kBN;
-    const int32_t* kinfo_src = has_win ? coord_kv_b : seg_kv_b;   // null with neither
-    const uint32_t my_coord = (has_win && row_valid) ? uint32_t(__ldg(coord_q_b + row)) : 0u;
-
-    float m_run = -INFINITY;   // running max of scale*log2(e)*s, the offset of P
-    float l_run = 0.f;         // running sum of P (fp32, before bf16 rounding)
-    int t = 0;
+    int T = 0;      // key tiles done by this CTA, over all units (barrier parities)
     bool ok = true;
-    for (int j = sched.tile(0, -1); j < n_kv; ++t, j = sched.tile(t, j)) {
-      bool masked;
-      if (listed) {
-        masked = (tile_list[t] >> (30 + qi)) & 1;
-      } else {
-        masked = (ragged_kv && j == p.n_kv_tiles - 1) || causal_partial(p, pair, qi, j) || has_win;
-        if (has_seg) {
-          const int4 ks = __ldg(sched.walk.kv_sum + j);
-          masked = masked || !(my_qs.z && ks.z && my_qs.x == ks.x);
-        }
-      }
-      const bool slow = masked || !(c > 0.f);
-      // A masked tile's key ids / coordinates: loads issued before the wait
-      // for S, so their latency hides behind it (warp-uniform: masked is the
-      // same for every row of a Q tile).
-      int32_t pre[4] = {0, 0, 0, 0};
-      if (masked && kinfo_src != nullptr) {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int x = j * kBN + lane + 32 * m;
-          if (x < p.S_kv) pre[m] = __ldg(kinfo_src + x);
-        }
-      }
-      VIDATTN_TR(1 + qi, t, 0);
-      ok = warp_wait_phase(s_full(qi), t & 1, abort_flag, p.err);
-      VIDATTN_TR(1 + qi, t, 1);
+    for (int u = blockIdx.x, k = 0; ok && u < u_end; u += u_step, ++k) {
+      const int* list;
+      int n_list;
+      ok = wait_list(k, &list, &n_list);
       if (!ok) break;
-      tc_fence_after();
-      if (masked && kinfo_src != nullptr) {
-        // the previous masked tile's mask was built before this point (the
-        // __syncwarp after it), so the slot is free
-#pragma unroll
-        for (int m = 0; m < 4; ++m) kinfo[lane + 32 * m] = pre[m];
-      }
-      // visible keys of this row: all of an unmasked tile; a masked tile's
-      // mask is built where it is used (the exact paths), from the slot
-      auto build_mask = [&](uint32_t (&mb)[4]) {
-        const int j0 = j * kBN;
-        const int n_valid = min(kBN, p.S_kv - j0);
-        const int n_lim =
-            p.causal ? max(0, min(n_valid, row + p.causal_off - j0 + 1)) : n_valid;
-        const WinRow wr = win_row(p, my_coord);
-        __syncwarp();
-        const int mode = has_win ? 2 : (has_seg ? 1 : 0);
-        const uint4 m =
-            kMaskFast ? tile_mask(kinfo, mode, my_seg, wr.s[0], wr.s[1], wr.s[2], p.win_size[0],
-                                  p.win_size[1], p.win_size[2], n_lim)
-                      : tile_mask_call(kinfo, mode, my_seg, wr.s[0], wr.s[1], wr.s[2],
-                                       p.win_size[0], p.win_size[1], p.win_size[2], n_lim);
-        __syncwarp();   // every lane has read the slot before it is refilled
-        mb[0] = m.x;
-        mb[1] = m.y;
-        mb[2] = m.z;
-        mb[3] = m.w;
-      };
+      const Unit x = decode_unit(p, u);
+      const int bh = x.b * p.H + x.h;
+      const int pair = x.pair;
+      const int row = pair * 2 * kBM + qi * kBM + r;
+      const bool row_valid = row < p.S_q;
+      // Values only masked tiles use (the row's id or coordinate, the keys'
+      // ids or coordinates) are read where they are used, from x.b and row,
+      // so that nothing more stays live across the tile loop.
+      int4 my_qs;
+      make_walk(p, x.b, pair, qi, &my_qs);
+      const UnitSched sched = unit_sched(p, x, list, n_list);
 
-      if constexpr (C::kSepP) {
-        // S row into registers, then S's columns are released to the MMA warp.
-        float s[kBN];
-        load_s_row(tS, s);
-        tc_fence_before();
-        mbar_arrive(s_free(qi));
-        VIDATTN_TR(1 + qi, t, 2);
-        uint32_t pk[2][32];
-        float rs = 0.f, alpha = 1.f;
-        bool rescale = false;
-        // running-offset path first (see the aliased-P branch below); the
-        // exact path works on the registers, since S may be overwritten now
-        bool exact = __any_sync(0xffffffffu, slow || (m_run == -INFINITY));
-        if (!exact) {
-          rs = exp_tile<kEmu>(s, c, m_run, pk);
-          exact = __any_sync(0xffffffffu, !(rs <= kStaleSumLimit));
+      float m_run = -INFINITY;   // running max of scale*log2(e)*s, the offset of P
+      float l_run = 0.f;         // running sum of P (fp32, before bf16 rounding)
+      int lt = 0;                // tiles of this unit done
+      int t = sched.t0;
+      for (int j = sched.tile(t, t - 1); j < sched.n_kv; ++t, ++lt, ++T, j = sched.tile(t, j)) {
+        bool masked;
+        if (list != nullptr) {
+          masked = (list[t] >> (30 + qi)) & 1;
+        } else {
+          masked = (ragged_kv && j == p.n_kv_tiles - 1) || causal_partial(p, pair, qi, j) || has_win;
+          if (has_seg) {
+            const int4 ks = __ldg(sched.walk.kv_sum + j);
+            masked = masked || !(my_qs.z && ks.z && my_qs.x == ks.x);
+          }
         }
-        if (exact) {
-          float tile_max;
-          if (!slow) {
-            tile_max = row_max(s) * c;
-          } else {
+        const bool slow = masked || !(c > 0.f);
+        // A masked tile's key ids / coordinates: loads issued before the wait
+        // for S, so their latency hides behind it (warp-uniform: masked is the
+        // same for every row of a Q tile).
+        int32_t pre[4] = {0, 0, 0, 0};
+        if (masked && has_sum) {
+          // the keys' ids or coordinates (tile summaries come with one or the other)
+          const int32_t* src = (has_win ? p.coord_kv : p.seg_kv) + static_cast<int64_t>(x.b) * p.S_kv;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int xk = j * kBN + lane + 32 * m;
+            if (xk < p.S_kv) pre[m] = __ldg(src + xk);
+          }
+        }
+        VIDATTN_TR(1 + qi, T, 0);
+        ok = warp_wait_phase(s_full(qi), uint32_t(T) & 1u, abort_flag, p.err);
+        VIDATTN_TR(1 + qi, T, 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (masked && has_sum) {
+          // the previous masked tile's mask was built before this point (the
+          // __syncwarp after it), so the slot is free
+#pragma unroll
+          for (int m = 0; m < 4; ++m) kinfo[lane + 32 * m] = pre[m];
+        }
+        // visible keys of this row: all of an unmasked tile; a masked tile's
+        // mask is built where it is used (the exact paths), from the slot
+        auto build_mask = [&](uint32_t (&mb)[4]) {
+          const int j0 = j * kBN;
+          const int n_valid = min(kBN, p.S_kv - j0);
+          const int n_lim =
+              p.causal ? max(0, min(n_valid, row + p.causal_off - j0 + 1)) : n_valid;
+          const int64_t qrow = static_cast<int64_t>(x.b) * p.S_q + row;
+          const int my_seg = (has_seg && row_valid) ? __ldg(p.seg_q + qrow) : 0;
+          const uint32_t my_coord = (has_win && row_valid) ? uint32_t(__ldg(p.coord_q + qrow)) : 0u;
+          const WinRow wr = win_row(p, my_coord);
+          __syncwarp();
+          const int mode = has_win ? 2 : (has_seg ? 1 : 0);
+          const uint4 m =
+              kMaskFast ? tile_mask(kinfo, mode, my_seg, wr.s[0], wr.s[1], wr.s[2], p.win_size[0],
+                                    p.win_size[1], p.win_size[2], n_lim)
+                        : tile_mask_call(kinfo, mode, my_seg, wr.s[0], wr.s[1], wr.s[2],
+                                         p.win_size[0], p.win_size[1], p.win_size[2], n_lim);
+          __syncwarp();   // every lane has read the slot before it is refilled
+          mb[0] = m.x;
+          mb[1] = m.y;
+          mb[2] = m.z;
+          mb[3] = m.w;
+        };
+
+        if constexpr (C::kSepP) {
+          // S row into registers; S's columns go back to the MMA warp once
+          // this tile's P is computed (P has columns of its own).
+          float s[kBN];
+          load_s_row(tS, s);
+          VIDATTN_TR(1 + qi, T, 2);
+          uint32_t pk[2][32];
+          float rs = 0.f, alpha = 1.f;
+          bool rescale = false;
+          // running-offset path first (see the aliased-P branch below); its
+          // exponentials consume the S registers as they go, so the exact
+          // path reads S from tensor memory again (still intact: s_free
+          // comes after)
+          bool exact = __any_sync(0xffffffffu, slow || (m_run == -INFINITY));
+          if (!exact) {
+            rs = exp_tile<kEmu>(s, c, m_run, pk);
+            exact = __any_sync(0xffffffffu, !(rs <= kStaleSumLimit));
+          }
+          if (exact) {
+            // the mask first: no S register is live across its call
             uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
             if (masked) build_mask(mb);
-            float mx = -INFINITY;
+            load_s_row(tS, s);
+            float tile_max;
+            if (!slow) {
+              tile_max = row_max(s) * c;
+            } else {
+              float mx = -INFINITY;
 #pragma unroll
-            for (int x = 0; x < kBN; ++x) {
-              const bool valid = (mb[x >> 5] >> (x & 31)) & 1u;
-              s[x] = valid ? s[x] * c : -INFINITY;
-              mx = fmaxf(mx, s[x]);
+              for (int xk = 0; xk < kBN; ++xk) {
+                const bool valid = (mb[xk >> 5] >> (xk & 31)) & 1u;
+                s[xk] = valid ? s[xk] * c : -INFINITY;
+                mx = fmaxf(mx, s[xk]);
+              }
+              tile_max = mx;
             }
-            tile_max = mx;
-          }
-          const float m_new = fmaxf(m_run, tile_max);
-          rescale = (m_new - m_run) > kRescaleThreshold;
-          if (rescale) {
-            alpha = ex2(m_run - m_new);
-            m_run = m_new;
-          }
-          const float msub = (m_run == -INFINITY) ? 0.f : m_run;
-          if (!slow) {
-            rs = exp_tile<kEmu>(s, c, msub, pk);
-          } else {
-            float r4[4] = {0.f, 0.f, 0.f, 0.f};
+            const float m_new = fmaxf(m_run, tile_max);
+            rescale = (m_new - m_run) > kRescaleThreshold;
+            if (rescale) {
+              alpha = ex2(m_run - m_new);
+              m_run = m_new;
+            }
+            const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+            if (!slow) {
+              rs = exp_tile<kEmu>(s, c, msub, pk);
+            } else {
+              float r4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int x = 0; x < kBN; x += 2) {
-              const float e0 = ex2(s[x] - msub);
-              const float e1 = ex2(s[x + 1] - msub);
-              r4[(x >> 1) & 3] += e0 + e1;
-              pk[x >> 6][(x >> 1) & 31] = pack_bf16x2(e0, e1);
+              for (int xk = 0; xk < kBN; xk += 2) {
+                const float e0 = ex2(s[xk] - msub);
+                const float e1 = ex2(s[xk + 1] - msub);
+                r4[(xk >> 1) & 3] += e0 + e1;
+                pk[xk >> 6][(xk >> 1) & 31] = pack_bf16x2(e0, e1);
+              }
+              rs = (r4[0] + r4[1]) + (r4[2] + r4[3]);
             }
-            rs = (r4[0] + r4[1]) + (r4[2] + r4[3]);
           }
-        }
-        l_run = l_run * alpha + rs;
-        VIDATTN_TR(1 + qi, t, 3);
-        // The previous P V of this tile has read P's columns and finished
-        // accumulating O: P may be overwritten and O rescaled.
-        if (t > 0) {
-          ok = warp_wait_phase(o_full(qi), (t - 1) & 1, abort_flag, p.err);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        VIDATTN_TR(1 + qi, t, 4);
-        tmem_st32(tP, pk[0]);
-        tmem_st32(tP + 32, pk[1]);
-        if (__any_sync(0xffffffffu, rescale && t > 0)) {
+          tc_fence_before();
+          mbar_arrive(s_free(qi));
+          l_run = l_run * alpha + rs;
+          VIDATTN_TR(1 + qi, T, 3);
+          // The previous P V of this tile has read P's columns and finished
+          // accumulating O: P may be overwritten and O rescaled.  (Before a
+          // unit's first tile the previous unit's epilogue waited for it.)
+          if (lt > 0) {
+            ok = warp_wait_phase(o_full(qi), uint32_t(T - 1) & 1u, abort_flag, p.err);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          VIDATTN_TR(1 + qi, T, 4);
+          tmem_st32(tP, pk[0]);
+          tmem_st32(tP + 32, pk[1]);
+          if (__any_sync(0xffffffffu, rescale && lt > 0)) {
 #pragma unroll 1
-          for (int k = 0; k < D / 32; ++k) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * k, o);
-            tmem_ld_wait();
-            reg_fence(o);
+            for (int kk = 0; kk < D / 32; ++kk) {
+              uint32_t o[32];
+              tmem_ld32(tO + 32 * kk, o);
+              tmem_ld_wait();
+              reg_fence(o);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(tO + 32 * k, o);
-          }
-        }
-        tmem_st_wait();
-      } else {
-        // P = 2^(c*s - m_run) for this tile, rounded to bf16 into pk; rs = its
-        // row sum in fp32.  Softmax does not depend on the offset m_run, so after
-        // a row's first tile the running offset is used as it stands ("stale"
-        // path, no max).  The offset only has to keep every exponential finite:
-        // if the tile's sum exceeds 2^32 the row takes the exact path instead,
-        // which computes the tile max, moves m_run up (rescaling O and l), and
-        // redoes the exponentials.  The exact path also serves masked tiles,
-        // a row's first tile, and scale <= 0.
-        float rs = 0.f, alpha = 1.f;
-        bool rescale = false;
-        // warp-uniform choice: the stale path only if every row of the warp
-        // can take it (with kMaskFast masked tiles too: hidden keys get p = 0)
-        bool exact = __any_sync(0xffffffffu, (kMaskFast ? !(c > 0.f) : slow) || (m_run == -INFINITY));
-        if (!exact) {
-          // a masked tile: its mask first (before S occupies the registers),
-          // then hidden keys' scores become -inf, i.e. p = 0 (the FMA-pipe
-          // exponential clamps at 2^-125, far below bf16 P's resolution
-          // against the row sum, which includes the row's running maximum)
-          uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
-          if (kMaskFast && masked) build_mask(mb);
-          float s[kBN];
-          uint32_t pk[2][32];
-          load_s_row(tS, s);
-          VIDATTN_TR(1 + qi, t, 2);
-          if (kMaskFast && masked) {
-#pragma unroll
-            for (int x = 0; x < kBN; ++x)
-              s[x] = ((mb[x >> 5] >> (x & 31)) & 1u) ? s[x] : -INFINITY;
-          }
-          rs = exp_tile<kEmu>(s, c, m_run, pk);
-          VIDATTN_TR(1 + qi, t, 3);
-          exact = __any_sync(0xffffffffu, !(rs <= kStaleSumLimit));
-          if (!exact) {
-            tmem_st32(tS, pk[0]);
-            tmem_st32(tS + 32, pk[1]);
-          }
-        }
-        if (exact) {
-          // Two passes over the tile, 32 columns at a time, straight from
-          // tensor memory (S is intact: no P has been written yet).  The sum
-          // restarts: a failed running-offset attempt leaves its sum in rs.
-          rs = 0.f;
-          uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
-          if (masked) build_mask(mb);
-          // this chunk's 32 mask bits (k is a runtime index: select, don't index)
-          auto chunk_bits = [&](int k) {
-            return k == 0 ? mb[0] : (k == 1 ? mb[1] : (k == 2 ? mb[2] : mb[3]));
-          };
-          float mx = -INFINITY;
-  #pragma unroll 1
-          for (int k = 0; k < 4; ++k) {
-            uint32_t r[32];
-            tmem_ld32(tS + 32 * k, r);
-            const uint32_t mk = chunk_bits(k);
-            tmem_ld_wait();
-            reg_fence(r);
-  #pragma unroll
-            for (int x = 0; x < 32; ++x)
-              mx = fmaxf(mx, ((mk >> x) & 1u) ? __uint_as_float(r[x]) * c : -INFINITY);
-          }
-          const float m_new = fmaxf(m_run, mx);
-          rescale = (m_new - m_run) > kRescaleThreshold;   // false for -inf - -inf
-          if (rescale) {
-            alpha = ex2(m_run - m_new);   // 0 when m_run is -inf
-            m_run = m_new;
-          }
-          const float msub = (m_run == -INFINITY) ? 0.f : m_run;
-          // P chunk k (keys 32k..32k+31) lands in columns [16k, 16k+16), which
-          // hold S columns already read: chunks are processed in order.
-  #pragma unroll 1
-          for (int k = 0; k < 4; ++k) {
-            uint32_t r[32], w[16];
-            tmem_ld32(tS + 32 * k, r);
-            const uint32_t mk = chunk_bits(k);
-            tmem_ld_wait();
-            reg_fence(r);
-  #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const float e0 = ((mk >> x) & 1u) ? ex2(__uint_as_float(r[x]) * c - msub) : 0.f;
-              const float e1 =
-                  ((mk >> (x + 1)) & 1u) ? ex2(__uint_as_float(r[x + 1]) * c - msub) : 0.f;
-              rs += e0 + e1;
-              w[x >> 1] = pack_bf16x2(e0, e1);
+              for (int xk = 0; xk < 32; ++xk)
+                o[xk] = __float_as_uint(__uint_as_float(o[xk]) * alpha);
+              tmem_st32(tO + 32 * kk, o);
             }
-            tmem_st16(tS + 16 * k, w);
-          }
-        }
-        l_run = l_run * alpha + rs;
-        tmem_st_wait();
-        // Rescale this tile's O rows before the next P.V accumulates into them.
-        if (__any_sync(0xffffffffu, rescale && t > 0)) {
-          ok = warp_wait_phase(o_full(qi), (t - 1) & 1, abort_flag, p.err);
-          if (!ok) break;
-          tc_fence_after();
-  #pragma unroll 1
-          for (int k = 0; k < D / 32; ++k) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * k, o);
-            tmem_ld_wait();
-            reg_fence(o);
-  #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(tO + 32 * k, o);
           }
           tmem_st_wait();
+        } else {
+          // P = 2^(c*s - m_run) for this tile, rounded to bf16 into pk; rs = its
+          // row sum in fp32.  Softmax does not depend on the offset m_run, so after
+          // a row's first tile the running offset is used as it stands ("stale"
+          // path, no max).  The offset only has to keep every exponential finite:
+          // if the tile's sum exceeds 2^32 the row takes the exact path instead,
+          // which computes the tile max, moves m_run up (rescaling O and l), and
+          // redoes the exponentials.  The exact path also serves masked tiles,
+          // a row's first tile, and scale <= 0.
+          float rs = 0.f, alpha = 1.f;
+          bool rescale = false;
+          // warp-uniform choice: the stale path only if every row of the warp
+          // can take it (with kMaskFast masked tiles too: hidden keys get p = 0)
+          bool exact =
+              __any_sync(0xffffffffu, (kMaskFast ? !(c > 0.f) : slow) || (m_run == -INFINITY));
+          if (!exact) {
+            // a masked tile: its mask first (before S occupies the registers),
+            // then hidden keys' scores become -inf, i.e. p = 0 (the FMA-pipe
+            // exponential clamps at 2^-125, far below bf16 P's resolution
+            // against the row sum, which includes the row's running maximum)
+            uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+            if (kMaskFast && masked) build_mask(mb);
+            float s[kBN];
+            uint32_t pk[2][32];
+            load_s_row(tS, s);
+            VIDATTN_TR(1 + qi, T, 2);
+            if (kMaskFast && masked) {
+#pragma unroll
+              for (int xk = 0; xk < kBN; ++xk)
+                s[xk] = ((mb[xk >> 5] >> (xk & 31)) & 1u) ? s[xk] : -INFINITY;
+            }
+            rs = exp_tile<kEmu>(s, c, m_run, pk);
+            VIDATTN_TR(1 + qi, T, 3);
+            exact = __any_sync(0xffffffffu, !(rs <= kStaleSumLimit));
+            if (!exact) {
+              tmem_st32(tS, pk[0]);
+              tmem_st32(tS + 32, pk[1]);
+            }
+          }
+          if (exact) {
+            // Two passes over the tile, 32 columns at a time, straight from
+            // tensor memory (S is intact: no P has been written yet).  The sum
+            // restarts: a failed running-offset attempt leaves its sum in rs.
+            rs = 0.f;
+            uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+            if (masked) build_mask(mb);
+            // this chunk's 32 mask bits (kk is a runtime index: select, don't index)
+            auto chunk_bits = [&](int kk) {
+              return kk == 0 ? mb[0] : (kk == 1 ? mb[1] : (kk == 2 ? mb[2] : mb[3]));
+            };
+            float mx = -INFINITY;
+#pragma unroll 1
+            for (int kk = 0; kk < 4; ++kk) {
+              uint32_t rr[32];
+              tmem_ld32(tS + 32 * kk, rr);
+              const uint32_t mk = chunk_bits(kk);
+              tmem_ld_wait();
+              reg_fence(rr);
+#pragma unroll
+              for (int xk = 0; xk < 32; ++xk)
+                mx = fmaxf(mx, ((mk >> xk) & 1u) ? __uint_as_float(rr[xk]) * c : -INFINITY);
+            }
+            const float m_new = fmaxf(m_run, mx);
+            rescale = (m_new - m_run) > kRescaleThreshold;   // false for -inf - -inf
+            if (rescale) {
+              alpha = ex2(m_run - m_new);   // 0 when m_run is -inf
+              m_run = m_new;
+            }
+            const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+            // P chunk kk (keys 32kk..32kk+31) lands in columns [16kk, 16kk+16),
+            // which hold S columns already read: chunks are processed in order.
+#pragma unroll 1
+            for (int kk = 0; kk < 4; ++kk) {
+              uint32_t rr[32], wv[16];
+              tmem_ld32(tS + 32 * kk, rr);
+              const uint32_t mk = chunk_bits(kk);
+              tmem_ld_wait();
+              reg_fence(rr);
+#pragma unroll
+              for (int xk = 0; xk < 32; xk += 2) {
+                const float e0 = ((mk >> xk) & 1u) ? ex2(__uint_as_float(rr[xk]) * c - msub) : 0.f;
+                const float e1 =
+                    ((mk >> (xk + 1)) & 1u) ? ex2(__uint_as_float(rr[xk + 1]) * c - msub) : 0.f;
+                rs += e0 + e1;
+                wv[xk >> 1] = pack_bf16x2(e0, e1);
+              }
+              tmem_st16(tS + 16 * kk, wv);
+            }
+          }
+          l_run = l_run * alpha + rs;
+          tmem_st_wait();
+          // Rescale this tile's O rows before the next P.V accumulates into them.
+          if (__any_sync(0xffffffffu, rescale && lt > 0)) {
+            ok = warp_wait_phase(o_full(qi), uint32_t(T - 1) & 1u, abort_flag, p.err);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int kk = 0; kk < D / 32; ++kk) {
+              uint32_t o[32];
+              tmem_ld32(tO + 32 * kk, o);
+              tmem_ld_wait();
+              reg_fence(o);
+#pragma unroll
+              for (int xk = 0; xk < 32; ++xk)
+                o[xk] = __float_as_uint(__uint_as_float(o[xk]) * alpha);
+              tmem_st32(tO + 32 * kk, o);
+            }
+            tmem_st_wait();
+          }
         }
+        tc_fence_before();
+        mbar_arrive(p_full(qi));
+        VIDATTN_TR(1 + qi, T, 5);
       }
-      tc_fence_before();
-      mbar_arrive(p_full(qi));
-      VIDATTN_TR(1 + qi, t, 5);
-    }
+      if (!ok) break;
+      release_list(k);
 
-    // ------------------------------------------------------------ epilogue
-    if (ok) {
-      if (t > 0) {
-        ok = warp_wait_phase(o_full(qi), (t - 1) & 1, abort_flag, p.err);
+      // ---------------------------------------------------------- epilogue
+      // O of the unit's last tile is complete once its P V has run.  The
+      // next unit's first P V overwrites O only after this warpgroup's
+      // p_full arrival for that tile, which follows these reads.
+      if (lt > 0) {
+        ok = warp_wait_phase(o_full(qi), uint32_t(T - 1) & 1u, abort_flag, p.err);
+        if (!ok) break;
         tc_fence_after();
       }
       const bool empty = !(l_run > 0.f);
       const float inv_l = empty ? 0.f : 1.f / l_run;
-      const int64_t orow = static_cast<int64_t>(bh) * p.S_q + row;
-      uint16_t* out_row = p.out + orow * D;
+      const float lse_row = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+      if constexpr (!kSplit) {
+        const int64_t orow = static_cast<int64_t>(bh) * p.S_q + row;
+        uint16_t* out_row = p.out + orow * D;
 #pragma unroll 1
-      for (int k = 0; k < D / 32; ++k) {
-        uint32_t o[32];
-        if (t > 0 && ok) {
-          tmem_ld32(tO + 32 * k, o);
-          tmem_ld_wait();
-          reg_fence(o);
-        } else {
+        for (int kk = 0; kk < D / 32; ++kk) {
+          uint32_t o[32];
+          if (lt > 0) {
+            tmem_ld32(tO + 32 * kk, o);
+            tmem_ld_wait();
+            reg_fence(o);
+          } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = 0u;
+            for (int xk = 0; xk < 32; ++xk) o[xk] = 0u;
+          }
+          uint32_t wv[16];
+#pragma unroll
+          for (int xk = 0; xk < 16; ++xk)
+            wv[xk] = pack_bf16x2(__uint_as_float(o[2 * xk]) * inv_l,
+                                 __uint_as_float(o[2 * xk + 1]) * inv_l);
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(out_row + 32 * kk);
+#pragma unroll
+            for (int xk = 0; xk < 4; ++xk)
+              dst[xk] = make_uint4(wv[4 * xk], wv[4 * xk + 1], wv[4 * xk + 2], wv[4 * xk + 3]);
+          }
         }
-        uint32_t w[16];
+        if (row_valid) p.lse[orow] = lse_row;
+      } else {
+        // one key split of the row: O / l and the split's log-sum-exp in
+        // fp32, merged by split_combine_kernel
+        const int64_t prow = (static_cast<int64_t>(bh) * p.n_split + x.split) * p.S_q + row;
+        float* po = p.part_o + prow * D;
+#pragma unroll 1
+        for (int kk = 0; kk < D / 32; ++kk) {
+          uint32_t o[32];
+          if (lt > 0) {
+            tmem_ld32(tO + 32 * kk, o);
+            tmem_ld_wait();
+            reg_fence(o);
+          } else {
 #pragma unroll
-        for (int x = 0; x < 16; ++x)
-          w[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv_l, __uint_as_float(o[2 * x + 1]) * inv_l);
-        if (row_valid && ok) {
-          uint4* dst = reinterpret_cast<uint4*>(out_row + 32 * k);
+            for (int xk = 0; xk < 32; ++xk) o[xk] = 0u;
+          }
+          if (row_valid) {
+            float4* dst = reinterpret_cast<float4*>(po + 32 * kk);
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+            for (int xk = 0; xk < 8; ++xk)
+              dst[xk] = make_float4(__uint_as_float(o[4 * xk]) * inv_l,
+                                    __uint_as_float(o[4 * xk + 1]) * inv_l,
+                                    __uint_as_float(o[4 * xk + 2]) * inv_l,
+                                    __uint_as_float(o[4 * xk + 3]) * inv_l);
+          }
         }
+        if (row_valid) p.part_lse[prow] = lse_row;
       }
-      if (row_valid && ok)
-        p.lse[orow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994530942f;
     }
   }
 
@@ -1169,6 +1358,51 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
+}
+
+// Merges the key splits of a split launch: per query row, with lse_s and
+// O_s (O / l) of each split s, lse = log sum_s exp(lse_s) and
+// out = sum_s exp(lse_s - lse) O_s, rounded once to bf16.  A row no split
+// saw (every lse_s = -inf) gets out = 0, lse = -inf.  One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) split_combine_kernel(const float* __restrict__ part_o,
+                                                            const float* __restrict__ part_lse,
+                                                            uint16_t* __restrict__ out,
+                                                            float* __restrict__ lse, int S_q,
+                                                            int n_split, int64_t n_rows) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= n_rows) return;
+  const int64_t bh = w / S_q;
+  const int64_t row = w - bh * S_q;
+  constexpr int kPer = D / 32;   // columns per lane
+  float mx = -INFINITY;
+  for (int s = 0; s < n_split; ++s)
+    mx = fmaxf(mx, __ldg(part_lse + (bh * n_split + s) * S_q + row));
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float total = 0.f;
+  if (mx != -INFINITY) {
+    for (int s = 0; s < n_split; ++s) {
+      const int64_t prow = (bh * n_split + s) * S_q + row;
+      const float ls = __ldg(part_lse + prow);
+      if (ls == -INFINITY) continue;
+      const float wgt = exp2f((ls - mx) * 1.44269504088896341f);
+      total += wgt;
+      const float* po = part_o + prow * D + lane * kPer;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] += wgt * __ldg(po + e);
+    }
+  }
+  const float inv = total > 0.f ? 1.f / total : 0.f;
+  uint16_t* orow = out + w * D + lane * kPer;
+#pragma unroll
+  for (int e = 0; e < kPer; e += 2) {
+    const uint32_t pk = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+    *reinterpret_cast<uint32_t*>(orow + e) = pk;
+  }
+  if (lane == 0) lse[w] = total > 0.f ? mx + __logf(total) : -INFINITY;
 }
 
 }  // namespace vidattn

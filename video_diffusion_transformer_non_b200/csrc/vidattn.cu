@@ -42,7 +42,21 @@ static __device__ __align__(256) int4 g_noalloc_summaries[kNoAllocMaxTiles];
 
 namespace {
 
-constexpr const char* kVersion = "vidattn 0.1 (sm_100a: TMA + tcgen05/TMEM)";
+constexpr const char* kVersion = "vidattn 0.2 (sm_100a: TMA + tcgen05/TMEM, persistent)";
+
+// Split heuristic: a launch with fewer than kSplitFillSMs / 2 work units
+// (256-row query blocks x heads x batch) splits each block's key tiles into
+// up to kMaxAutoSplit ranges, enough to give about kSplitFillSMs units (the
+// B200's 148 SMs), at least kMinSplitTiles key tiles per split: below that
+// the merge kernel and each split's own first tile (two passes) cost more
+// than the parallelism gains (measured: the 512-token tiny workload takes
+// 16.7 us unsplit, 19.6 us in 2 splits, 18.2 us in 4).
+constexpr int kSplitFillSMs = 148;
+constexpr int kMaxAutoSplit = 16;
+constexpr int kMinSplitTiles = 8;
+// Persistent grid only for units of at most this many key tiles (below).
+constexpr int kPersistMaxTiles = 64;
+constexpr int kMaxSplit = 64;   // largest VIDATTN_SPLIT_KV request
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -79,6 +93,7 @@ struct DeviceInfo {
   uint32_t attrs_set = 0;   // bit (kernel variant index) once its smem limit is raised
   int* err = nullptr;       // device address of g_device_error on this device
   int rope_grid[4] = {};    // persistent grid of each rope3d variant (SMs x resident CTAs)
+  int sms = 0;              // streaming multiprocessors (the attention kernel's grid bound)
   // vidattn_fwd_host's copy streams (host-to-device, device-to-host) and
   // its second compute stream
   cudaStream_t copy_in = nullptr, copy_out = nullptr, compute2 = nullptr;
@@ -108,26 +123,42 @@ std::mutex g_map_mu;
 
 using FwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                            const FwdParams);
-// Variants of the attention kernel: head dim x exponentials per 16 keys on
-// the FMA pipe.
+// Variants of the attention kernel.  One CTA per unit, keys not split (the
+// common launch): head dim x exponentials per 16 keys on the FMA pipe.
 constexpr int kEmuChoices[] = {0, 2, 4, 6, 8};
 constexpr int kNumEmu = 5;
 template <int D>
 FwdKernel fwd_variant(int e) {
   switch (e) {
-    case 0: return vidattn_fwd_kernel<D, 0, false>;
-    case 1: return vidattn_fwd_kernel<D, 2, false>;
-    case 2: return vidattn_fwd_kernel<D, 4, false>;
-    case 3: return vidattn_fwd_kernel<D, 6, false>;
-    default: return vidattn_fwd_kernel<D, 8, false>;
+    case 0: return vidattn_fwd_kernel<D, 0, false, false, false>;
+    case 1: return vidattn_fwd_kernel<D, 2, false, false, false>;
+    case 2: return vidattn_fwd_kernel<D, 4, false, false, false>;
+    case 3: return vidattn_fwd_kernel<D, 6, false, false, false>;
+    default: return vidattn_fwd_kernel<D, 8, false, false, false>;
   }
+}
+// Persistent or split launches: the head dim's default share (4 of 16 at
+// D = 128, 2 of 16 at D = 64); a split launch is never persistent (it has
+// fewer units than SMs).
+FwdKernel fwd_persist_variant(int D) {
+  return D == 128 ? vidattn_fwd_kernel<128, 4, false, true, false>
+                  : vidattn_fwd_kernel<64, 2, false, true, false>;
+}
+FwdKernel fwd_split_variant(int D) {
+  return D == 128 ? vidattn_fwd_kernel<128, 4, false, false, true>
+                  : vidattn_fwd_kernel<64, 2, false, false, true>;
 }
 // 3D neighbourhood windows: masked tiles on the running-offset path (D = 128,
 // 2 of 16 exponentials on the FMA pipe: the mask work takes issue slots, and
 // 2 measured 3 % faster than 4 on the 11^3 window over the 480p volume);
-// D = 64 uses the default kernel.
-FwdKernel fwd_window_variant(int D) {
-  return D == 128 ? vidattn_fwd_kernel<128, 2, true> : vidattn_fwd_kernel<64, 2, false>;
+// D = 64 uses the default kernel.  Never persistent (a window call's units
+// span the whole key range of its tile summaries).
+FwdKernel fwd_window_variant(int D, bool split) {
+  if (split)
+    return D == 128 ? vidattn_fwd_kernel<128, 2, true, false, true>
+                    : vidattn_fwd_kernel<64, 2, false, false, true>;
+  return D == 128 ? vidattn_fwd_kernel<128, 2, true, false, false>
+                  : vidattn_fwd_kernel<64, 2, false, false, false>;
 }
 // Default share of exponentials moved off the MUFU unit (measured best on
 // B200: 4 of 16 at D = 128, 2 of 16 at D = 64, where the FMA-pipe version's
@@ -167,6 +198,8 @@ int ensure_device(int* dev_out) {
       return VIDATTN_ERR_CUDA;
     info.checked = true;
     info.ok = (major == 10 && minor == 0);
+    if (cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return VIDATTN_ERR_CUDA;
   }
   if (!info.ok) return VIDATTN_ERR_NO_DEVICE;
   if (info.err == nullptr) {
@@ -176,16 +209,20 @@ int ensure_device(int* dev_out) {
     info.err = static_cast<int*>(e);
   }
   if (info.attrs_set == 0) {
-    for (int e = 0; e < kNumEmu; ++e) {
-      if (cudaFuncSetAttribute(fwd_variant<64>(e), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               FwdCfg<64>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fwd_variant<128>(e), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               FwdCfg<128>::kSmemBytes) != cudaSuccess)
-        return VIDATTN_ERR_CUDA;
+    auto smem = [](FwdKernel k, int bytes) {
+      return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+             cudaSuccess;
+    };
+    bool ok = true;
+    for (int e = 0; e < kNumEmu; ++e)
+      ok = ok && smem(fwd_variant<64>(e), FwdCfg<64>::kSmemBytes) &&
+           smem(fwd_variant<128>(e), FwdCfg<128>::kSmemBytes);
+    for (int D : {64, 128}) {
+      const int bytes = D == 128 ? FwdCfg<128>::kSmemBytes : FwdCfg<64>::kSmemBytes;
+      ok = ok && smem(fwd_persist_variant(D), bytes) && smem(fwd_split_variant(D), bytes) &&
+           smem(fwd_window_variant(D, false), bytes) && smem(fwd_window_variant(D, true), bytes);
     }
-    if (cudaFuncSetAttribute(fwd_window_variant(128), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdCfg<128>::kSmemBytes) != cudaSuccess)
-      return VIDATTN_ERR_CUDA;
+    if (!ok) return VIDATTN_ERR_CUDA;
     info.attrs_set = 1;
   }
   return VIDATTN_OK;
@@ -231,6 +268,11 @@ int noalloc_scratch(int dev, int4** out) {
 int* device_error_word(int dev) {
   std::lock_guard<std::mutex> lk(g_mu);
   return g_devices[dev].err;
+}
+
+int device_sms(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_devices[dev].sms;
 }
 
 // Tensor map of bf16 [BH, S, D] at ptr on dev, from the cache when present.
@@ -283,11 +325,49 @@ struct WinSpec {
   int size[3], extent[3], clamped;
 };
 
+// Bytes of split partials (O / l and lse per row and split, fp32) for a launch.
+size_t split_bytes(int B, int H, int S_q, int D, int n_split) {
+  if (n_split <= 1) return 0;
+  return size_t(B) * H * n_split * S_q * (size_t(D) + 1) * 4;
+}
+
+// The launch's key splits: `requested` when the caller asks for a number
+// (VIDATTN_SPLIT_KV), else the heuristic of vidattn_split_count.
+int choose_split(int B, int H, int S_q, int S_kv, bool global_walk, int requested) {
+  if (S_q <= 0 || S_kv <= 0 || global_walk) return 1;
+  if (requested > 0) return requested;
+  const int64_t units = int64_t(B) * H * ((S_q + 2 * kBM - 1) / (2 * kBM));
+  if (units * 2 >= kSplitFillSMs) return 1;
+  const int n_kv = (S_kv + kBN - 1) / kBN;
+  int64_t want = (kSplitFillSMs + units - 1) / units;
+  if (want > n_kv / kMinSplitTiles) want = n_kv / kMinSplitTiles;
+  if (want > kMaxAutoSplit) want = kMaxAutoSplit;
+  return want < 1 ? 1 : int(want);
+}
+
+// Persistent grid or one CTA per unit (unsplit launches).  Persistence
+// overlaps a unit's epilogue with the next unit's loads and first Q K^T,
+// which pays when units are short: measured at D = 128 with more units than
+// SMs, +13 % at 4 key tiles per unit, +9 % at 8, +6 % at 16, +3 % at 32,
+// +1 % at 64; at D = 64 (16 tiles) nothing.  On long units the hardware's
+// dynamic placement of one CTA per unit balances the SMs better than the
+// static round-robin (the 480p and 720p workloads lose 1-2 % persistent).
+// VIDATTN_PERSIST=0/1 overrides, for experiments.
+bool use_persistent(int64_t n_units, int sms, int n_kv_tiles, int D) {
+  static const int forced = [] {
+    const char* e = getenv("VIDATTN_PERSIST");
+    return e ? (atoi(e) != 0 ? 1 : 0) : -1;
+  }();
+  if (forced >= 0) return forced == 1;
+  return D == 128 && n_units > sms && n_kv_tiles <= kPersistMaxTiles;
+}
+
 template <int D>
 int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32_t* seg_q,
                const int32_t* seg_kv, const int4* q_sum, const int4* kv_sum, void* out,
                float* lse, int B, int H, int S_q, int S_kv, float scale, cudaStream_t stream,
-               int flags = 0, const WinSpec* win = nullptr) {
+               int flags = 0, const WinSpec* win = nullptr, int n_split = 1,
+               float* part = nullptr) {
   CUtensorMap tq, tk, tv;
   const int64_t BH = int64_t(B) * H;
   // With no keys the K/V maps are never read; they are encoded over q.
@@ -311,6 +391,15 @@ int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32
   p.n_kv_tiles = (S_kv + kBN - 1) / kBN;
   p.causal = (flags & VIDATTN_CAUSAL) ? 1 : 0;
   p.causal_off = S_kv - S_q;
+  p.n_pairs = (S_q + 2 * kBM - 1) / (2 * kBM);
+  p.n_split = n_split;
+  const int64_t n_units = int64_t(B) * H * p.n_pairs * n_split;
+  if (n_units > INT_MAX) return VIDATTN_ERR_BAD_SHAPE;
+  p.n_units = int(n_units);
+  if (n_split > 1) {
+    p.part_o = part;
+    p.part_lse = part + size_t(B) * H * n_split * S_q * D;
+  }
   if (win) {
     p.coord_q = win->coord_q;
     p.coord_kv = win->coord_kv;
@@ -324,10 +413,25 @@ int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32
 #ifdef VIDATTN_TRACE
   p.trace = g_trace;
 #endif
-  dim3 grid((S_q + 2 * kBM - 1) / (2 * kBM), H, B);
-  FwdKernel kernel = win ? fwd_window_variant(D) : fwd_variant<D>(emu_index(D));
+  // persistent: at most one CTA per SM (tensor and shared memory are sized
+  // for one), each looping over units; else one CTA per unit
+  const int sms = device_sms(dev);
+  const bool persist = !win && n_split == 1 && use_persistent(n_units, sms, p.n_kv_tiles, D);
+  const int grid = int(persist ? (n_units > sms ? sms : n_units) : n_units);
+  FwdKernel kernel = win ? fwd_window_variant(D, n_split > 1)
+                         : (n_split > 1 ? fwd_split_variant(D)
+                                        : (persist ? fwd_persist_variant(D)
+                                                   : fwd_variant<D>(emu_index(D))));
   kernel<<<grid, kFwdThreads, FwdCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? VIDATTN_OK : VIDATTN_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
+  if (n_split > 1) {
+    const int64_t rows = int64_t(B) * H * S_q;
+    const int64_t blocks = (rows + 7) / 8;   // 8 warps, one row each
+    split_combine_kernel<D><<<unsigned(blocks), 256, 0, stream>>>(
+        p.part_o, p.part_lse, static_cast<uint16_t*>(out), lse, S_q, n_split, rows);
+    if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
+  }
+  return VIDATTN_OK;
 }
 
 // The streams of vidattn_fwd_host on device dev (created on first use).
@@ -435,13 +539,22 @@ VIDATTN_API const char* vidattn_status_string(int status) {
   }
 }
 
+VIDATTN_API int vidattn_split_count(const int32_t* seg_q, int B, int H, int S_q, int S_kv,
+                                    int flags) {
+  if (B < 1 || H < 1 || S_q < 1 || S_kv < 0) return 0;
+  const int requested = (flags >> 8) & 0xFF;
+  if (requested > kMaxSplit) return 0;
+  const bool global_walk = seg_q != nullptr && (S_kv + kBN - 1) / kBN > kMaxListedTiles;
+  return choose_split(B, H, S_q, S_kv, global_walk, requested);
+}
+
 VIDATTN_API int vidattn_kernels_per_call(const int32_t* seg_q, const int32_t* seg_kv, int B,
-                                         int H, int S_q, int S_kv, int D) {
+                                         int H, int S_q, int S_kv, int D, int flags) {
   (void)seg_kv;
-  (void)S_kv;
   (void)D;
   if (B < 1 || H < 1 || S_q < 1) return 0;
-  return seg_q ? 2 : 1;
+  const int n_split = vidattn_split_count(seg_q, B, H, S_q, S_kv, flags);
+  return (seg_q ? 2 : 1) + (n_split > 1 ? 1 : 0);
 }
 
 VIDATTN_API int vidattn_fwd(const void* q, const void* k, const void* v, const int32_t* seg_q,
@@ -454,7 +567,8 @@ VIDATTN_API int vidattn_fwd_ex(const void* q, const void* k, const void* v,
                                const int32_t* seg_q, const int32_t* seg_kv, void* out, float* lse,
                                int B, int H, int S_q, int S_kv, int D, float scale, int flags,
                                vidattn_stream_t stream_) {
-  if (flags & ~VIDATTN_CAUSAL) return VIDATTN_ERR_BAD_SHAPE;
+  if (flags & ~(VIDATTN_CAUSAL | VIDATTN_SPLIT_KV(0xFF))) return VIDATTN_ERR_BAD_SHAPE;
+  if (((flags >> 8) & 0xFF) > kMaxSplit) return VIDATTN_ERR_BAD_SHAPE;
   int st = check_args(q, k, v, seg_q, seg_kv, out, lse, B, H, S_q, S_kv, D);
   if (st != VIDATTN_OK) return st;
   if (!std::isfinite(scale)) return VIDATTN_ERR_BAD_SHAPE;
@@ -464,26 +578,36 @@ VIDATTN_API int vidattn_fwd_ex(const void* q, const void* k, const void* v,
   st = ensure_device(&dev);
   if (st != VIDATTN_OK) return st;
 
+  // scratch: the segment summaries, then (split launches) the partials
+  const int n_split = vidattn_split_count(seg_q, B, H, S_q, S_kv, flags);
+  const int nq = (S_q + kSegTile - 1) / kSegTile;
+  const int nk = (S_kv + kSegTile - 1) / kSegTile;
+  const size_t sum_bytes =
+      seg_q ? (sizeof(int4) * size_t(B) * (size_t(nq) + size_t(nk)) + 255) & ~size_t(255) : 0;
+  const size_t part_bytes = split_bytes(B, H, S_q, D, n_split);
+  char* buf = nullptr;
+  if (sum_bytes + part_bytes > 0) {
+    buf = static_cast<char*>(scratch_for(dev, stream, sum_bytes + part_bytes));
+    if (!buf) return VIDATTN_ERR_CUDA;
+  }
   const int4* q_sum = nullptr;
   const int4* kv_sum = nullptr;
   if (seg_q) {
-    const int nq = (S_q + kSegTile - 1) / kSegTile;
-    const int nk = (S_kv + kSegTile - 1) / kSegTile;
-    const size_t bytes = sizeof(int4) * size_t(B) * (size_t(nq) + size_t(nk));
-    int4* buf = static_cast<int4*>(scratch_for(dev, stream, bytes));
-    if (!buf) return VIDATTN_ERR_CUDA;
-    q_sum = buf;
-    kv_sum = buf + size_t(B) * nq;
+    int4* sums = reinterpret_cast<int4*>(buf);
+    q_sum = sums;
+    kv_sum = sums + size_t(B) * nq;
     dim3 grid(nq > nk ? nq : nk, B, 2);
-    seg_tile_classify_kernel<<<grid, 128, 0, stream>>>(seg_q, seg_kv, const_cast<int4*>(q_sum),
-                                                       const_cast<int4*>(kv_sum), S_q, S_kv);
+    seg_tile_classify_kernel<<<grid, 128, 0, stream>>>(seg_q, seg_kv, sums, sums + size_t(B) * nq,
+                                                       S_q, S_kv);
     if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
   }
+  float* part = part_bytes ? reinterpret_cast<float*>(buf + sum_bytes) : nullptr;
+  const int attn_flags = flags & VIDATTN_CAUSAL;
   if (D == 64)
-    return launch_fwd<64>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
-                          stream, flags);
-  return launch_fwd<128>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv, scale,
-                         stream, flags);
+    return launch_fwd<64>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv,
+                          scale, stream, attn_flags, nullptr, n_split, part);
+  return launch_fwd<128>(dev, q, k, v, seg_q, seg_kv, q_sum, kv_sum, out, lse, B, H, S_q, S_kv,
+                         scale, stream, attn_flags, nullptr, n_split, part);
 }
 
 VIDATTN_API int vidattn_fwd_window(const void* q, const void* k, const void* v,
@@ -512,21 +636,25 @@ VIDATTN_API int vidattn_fwd_window(const void* q, const void* k, const void* v,
 
   const int nq = (S_q + kSegTile - 1) / kSegTile;
   const int nk = (S_kv + kSegTile - 1) / kSegTile;
-  const size_t bytes = sizeof(int4) * size_t(B) * (size_t(nq) + size_t(nk > 0 ? nk : 1));
-  int4* buf = static_cast<int4*>(scratch_for(dev, stream, bytes));
+  const int n_split = choose_split(B, H, S_q, S_kv, false, 0);
+  const size_t box_bytes =
+      (sizeof(int4) * size_t(B) * (size_t(nq) + size_t(nk > 0 ? nk : 1)) + 255) & ~size_t(255);
+  const size_t part_bytes = split_bytes(B, H, S_q, D, n_split);
+  char* buf = static_cast<char*>(scratch_for(dev, stream, box_bytes + part_bytes));
   if (!buf) return VIDATTN_ERR_CUDA;
-  int4* q_box = buf;
-  int4* kv_box = buf + size_t(B) * nq;
+  int4* q_box = reinterpret_cast<int4*>(buf);
+  int4* kv_box = q_box + size_t(B) * nq;
   dim3 grid(nq > nk ? nq : nk, B, 2);
   win_tile_bbox_kernel<<<grid, 128, 0, stream>>>(coord_q, coord_kv, q_box, kv_box, S_q, S_kv);
   if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
   WinSpec win{coord_q, coord_kv, {win_t, win_h, win_w}, {T, Hg, Wg},
               (flags & VIDATTN_WINDOW_CLAMPED) ? 1 : 0};
+  float* part = part_bytes ? reinterpret_cast<float*>(buf + box_bytes) : nullptr;
   if (D == 64)
     return launch_fwd<64>(dev, q, k, v, nullptr, nullptr, q_box, kv_box, out, lse, B, H, S_q, S_kv,
-                          scale, stream, 0, &win);
+                          scale, stream, 0, &win, n_split, part);
   return launch_fwd<128>(dev, q, k, v, nullptr, nullptr, q_box, kv_box, out, lse, B, H, S_q, S_kv,
-                         scale, stream, 0, &win);
+                         scale, stream, 0, &win, n_split, part);
 }
 
 VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h_v,
@@ -577,6 +705,11 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
   cudaStream_t cin = nullptr, cout = nullptr, comp2 = nullptr;
   if (!host_streams(dev, &cin, &cout, &comp2)) return VIDATTN_ERR_CUDA;
   const int hc = (H + kPipelineChunks - 1) / kPipelineChunks;
+  // every chunk uses the whole call's key splits, so the result is the
+  // device entry point's bit for bit (a chunk alone has fewer work units
+  // and the heuristic could split it differently)
+  const int split_flag =
+      VIDATTN_SPLIT_KV(vidattn_split_count(d_seg_q, B, H, S_q, S_kv, 0));
   const size_t hq = size_t(S_q) * D * 2, hkv = size_t(S_kv) * D * 2, hl = size_t(S_q) * 4;
   auto ev = [](cudaEvent_t* e) {
     return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
@@ -619,9 +752,10 @@ VIDATTN_API int vidattn_fwd_host(const void* h_q, const void* h_k, const void* h
       cudaStream_t comp = (chunk++ & 1) ? comp2 : stream;
       ok = ok && cudaStreamWaitEvent(comp, in_done, 0) == cudaSuccess;
       if (ok) {
-        st = vidattn_fwd(dq, dk, dv, d_seg_q ? d_seg_q + size_t(b) * S_q : nullptr,
-                         d_seg_kv ? d_seg_kv + size_t(b) * S_kv : nullptr, dout, dl, 1, nh, S_q,
-                         S_kv, D, scale, reinterpret_cast<vidattn_stream_t>(comp));
+        st = vidattn_fwd_ex(dq, dk, dv, d_seg_q ? d_seg_q + size_t(b) * S_q : nullptr,
+                            d_seg_kv ? d_seg_kv + size_t(b) * S_kv : nullptr, dout, dl, 1, nh,
+                            S_q, S_kv, D, scale, split_flag,
+                            reinterpret_cast<vidattn_stream_t>(comp));
         ok = st == VIDATTN_OK;
       }
       ok = ok && cudaEventRecord(k_done, comp) == cudaSuccess &&
