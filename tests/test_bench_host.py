@@ -76,7 +76,8 @@ def test_committed_summaries_parse():
     for name in ("vidattn_fwd_kernel_d128__video_480p_h8.md", "rope3d_kernel_d128__video_480p.md",
                  "vidattn_fwd_kernel_d128__video_480p_causal_h8.md",
                  "vidattn_fwd_kernel_d64__cogvideox_joint_h8.md",
-                 "vidattn_fwd_kernel_d128__window_480p_h8.md"):
+                 "vidattn_fwd_kernel_d128__window_480p_h8.md",
+                 "vidattn_fwd_kernel_d128__video_720p_h8.md"):
         text = open(os.path.join(root, "profiles", name)).read()
         assert "kernel_sources_sha256:" in text and "traffic_bytes_per_full_launch:" in text
 
