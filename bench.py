@@ -539,10 +539,8 @@ def main(argv=None):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * (binding.kernels_per_call(
                 sq, sk, w.B, w.H, w.S_q, w.S_kv, w.D, flags) + (1 if use_rope or windowed else 0)),
-            "launch": {"grid_ctas": min(148, w.B * w.H * -(-w.S_q // 256) * binding.split_count(
-                           sq, w.B, w.H, w.S_q, w.S_kv, flags)),
-                       "key_splits": binding.split_count(sq, w.B, w.H, w.S_q, w.S_kv, flags),
-                       "persistent": True},
+            "launch": (None if windowed else
+                       binding.launch_plan(sq, w.B, w.H, w.S_q, w.S_kv, w.D, flags)),
             "rope3d": rope,
             "clocks": clocks,
         }

@@ -339,6 +339,17 @@ VIDATTN_API int vidattn_device_status(vidattn_stream_t stream);
 VIDATTN_API int vidattn_split_count(const int32_t* seg_q, int B, int H, int S_q, int S_kv,
                                     int flags);
 
+/* The launch a vidattn_fwd_ex call with these arguments would make on the
+ * current device (vidattn_split_count's splits, the persistent-grid choice
+ * above, and the attention kernel's grid): *grid_ctas CTAs, *key_splits
+ * key ranges per query block, *persistent 1 when each CTA loops over units.
+ * Queries the device's SM count (a CUDA call; no launch, no allocation).
+ * Returns VIDATTN_OK, or NULL / UNSUPPORTED_D / BAD_SHAPE (also for S_q < 1)
+ * / NO_DEVICE / CUDA errors, leaving the outputs unset. */
+VIDATTN_API int vidattn_launch_plan(const int32_t* seg_q, int B, int H, int S_q, int S_kv,
+                                    int D, int flags, int* grid_ctas, int* key_splits,
+                                    int* persistent);
+
 /* Number of kernels one vidattn_fwd_ex call with these arguments launches
  * (0 when there is nothing to compute): the attention kernel, plus the tile
  * classifier with segment ids, plus the merge of a split launch.

@@ -34,7 +34,8 @@ def test_header_declares_the_entry_points():
     assert {"vidattn_fwd", "vidattn_fwd_ex", "vidattn_fwd_host", "vidattn_status_string", "vidattn_device_status",
             "vidattn_rope3d", "vidattn_fwd_window",
             "vidattn_kernels_per_call", "vidattn_release", "vidattn_version",
-            "vidattn_selftest_timeout"} <= names
+            "vidattn_selftest_timeout", "vidattn_split_count", "vidattn_launch_plan",
+            "vidattn_fwd_noalloc"} <= names
     assert set(binding.exported_symbols()) == names
 
 
@@ -135,6 +136,22 @@ def test_split_heuristic(lib):
     assert sc(None, 1, 2, 512, 512, S(64)) == 64
     assert sc(None, 1, 2, 512, 512, S(65)) == 0       # above 64: invalid
     assert sc(None, 1, 2, 0, 512) == 0 and sc(None, 1, 2, 512, 0) == 1
+
+
+def test_launch_plan_argument_errors(lib):
+    """Argument errors come back before the device is touched; on a host
+    without an sm_100 GPU a valid query reports the missing device."""
+    import ctypes
+    g, k, pe = ctypes.c_int(-1), ctypes.c_int(-1), ctypes.c_int(-1)
+    refs = (ctypes.byref(g), ctypes.byref(k), ctypes.byref(pe))
+    assert lib.vidattn_launch_plan(None, 1, 2, 512, 512, 64, 0, None, refs[1], refs[2]) == NULL
+    assert lib.vidattn_launch_plan(None, 1, 2, 512, 512, 96, 0, *refs) == BAD_D
+    assert lib.vidattn_launch_plan(None, 1, 2, 512, 512, 64, 2, *refs) == BAD_SHAPE
+    assert lib.vidattn_launch_plan(None, 1, 2, 0, 512, 64, 0, *refs) == BAD_SHAPE
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.vidattn_launch_plan(None, 1, 2, 512, 512, 64, 0, *refs) != 0
+        assert (g.value, k.value, pe.value) == (-1, -1, -1)
 
 
 def test_selftest_argument_range(lib):

@@ -82,6 +82,21 @@ def test_auto_split_long_keys():
     assert float(d.max()) <= 1e-2 and float((l1 - l2).abs().max()) <= 1e-4
 
 
+def test_launch_plan_matches_the_heuristic():
+    """What vidattn_launch_plan reports for the workloads (148 SMs)."""
+    seg = np.zeros((2, 4389), np.int32)
+    sq = to_dev_i32(seg)
+    plan = binding.launch_plan
+    assert plan(None, 1, 2, 512, 512, 64) == dict(grid_ctas=4, key_splits=1, persistent=False)
+    assert plan(sq, 2, 12, 4389, 4389, 128) == dict(grid_ctas=148, key_splits=1, persistent=True)
+    assert plan(None, 1, 40, 32760, 32760, 128) == dict(grid_ctas=5120, key_splits=1,
+                                                        persistent=False)
+    assert plan(None, 2, 48, 17792, 17792, 64) == dict(grid_ctas=6720, key_splits=1,
+                                                       persistent=False)
+    assert plan(None, 1, 2, 512, 131072, 128) == dict(grid_ctas=64, key_splits=16,
+                                                      persistent=False)
+
+
 # ------------------------------------------------ persistent launches
 # Many short units (more than the 148 SMs, few key tiles each): the launch
 # is persistent, so every CTA carries its barrier phases, Q buffers and

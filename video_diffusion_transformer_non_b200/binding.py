@@ -58,6 +58,9 @@ def load_library():
     lib.vidattn_kernels_per_call.restype = i32
     lib.vidattn_split_count.argtypes = [p, i32, i32, i32, i32, i32]
     lib.vidattn_split_count.restype = i32
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.vidattn_launch_plan.argtypes = [p, i32, i32, i32, i32, i32, i32, ip, ip, ip]
+    lib.vidattn_launch_plan.restype = i32
     lib.vidattn_selftest_timeout.argtypes = [i32, p]
     lib.vidattn_selftest_timeout.restype = i32
     lib.vidattn_fwd_window.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, f32,
@@ -213,6 +216,18 @@ def split_count(seg_q, B, H, S_q, S_kv, flags=0) -> int:
     library's launch heuristic, or the VIDATTN_SPLIT_KV request in flags)."""
     return load_library().vidattn_split_count(_ptr(seg_q), int(B), int(H), int(S_q), int(S_kv),
                                               int(flags))
+
+
+def launch_plan(seg_q, B, H, S_q, S_kv, D, flags=0) -> dict:
+    """The launch a vidattn_fwd_ex call would make on the current device:
+    dict(grid_ctas, key_splits, persistent).  Raises on an error status."""
+    g, k, pe = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    st = load_library().vidattn_launch_plan(_ptr(seg_q), int(B), int(H), int(S_q), int(S_kv),
+                                            int(D), int(flags), ctypes.byref(g), ctypes.byref(k),
+                                            ctypes.byref(pe))
+    if st != VIDATTN_OK:
+        raise RuntimeError(f"vidattn_launch_plan: {status_string(st)}")
+    return dict(grid_ctas=g.value, key_splits=k.value, persistent=bool(pe.value))
 
 
 def VIDATTN_SPLIT_KV(n: int) -> int:

@@ -362,6 +362,11 @@ bool use_persistent(int64_t n_units, int sms, int n_kv_tiles, int D) {
   return D == 128 && n_units > sms && n_kv_tiles <= kPersistMaxTiles;
 }
 
+// CTAs of the attention launch: one per unit, or persistent with one per SM.
+int launch_grid(int64_t n_units, int sms, bool persist) {
+  return int(persist ? (n_units > sms ? sms : n_units) : n_units);
+}
+
 template <int D>
 int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32_t* seg_q,
                const int32_t* seg_kv, const int4* q_sum, const int4* kv_sum, void* out,
@@ -417,7 +422,7 @@ int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32
   // for one), each looping over units; else one CTA per unit
   const int sms = device_sms(dev);
   const bool persist = !win && n_split == 1 && use_persistent(n_units, sms, p.n_kv_tiles, D);
-  const int grid = int(persist ? (n_units > sms ? sms : n_units) : n_units);
+  const int grid = launch_grid(n_units, sms, persist);
   FwdKernel kernel = win ? fwd_window_variant(D, n_split > 1)
                          : (n_split > 1 ? fwd_split_variant(D)
                                         : (persist ? fwd_persist_variant(D)
@@ -546,6 +551,29 @@ VIDATTN_API int vidattn_split_count(const int32_t* seg_q, int B, int H, int S_q,
   if (requested > kMaxSplit) return 0;
   const bool global_walk = seg_q != nullptr && (S_kv + kBN - 1) / kBN > kMaxListedTiles;
   return choose_split(B, H, S_q, S_kv, global_walk, requested);
+}
+
+VIDATTN_API int vidattn_launch_plan(const int32_t* seg_q, int B, int H, int S_q, int S_kv,
+                                    int D, int flags, int* grid_ctas, int* key_splits,
+                                    int* persistent) {
+  if (!grid_ctas || !key_splits || !persistent) return VIDATTN_ERR_NULL;
+  if (D != 64 && D != 128) return VIDATTN_ERR_UNSUPPORTED_D;
+  if (flags & ~(VIDATTN_CAUSAL | VIDATTN_SPLIT_KV(0xFF))) return VIDATTN_ERR_BAD_SHAPE;
+  const int n_split = vidattn_split_count(seg_q, B, H, S_q, S_kv, flags);
+  if (n_split < 1) return VIDATTN_ERR_BAD_SHAPE;
+  int dev = 0;
+  const int st = ensure_device(&dev);
+  if (st != VIDATTN_OK) return st;
+  const int64_t n_units =
+      int64_t(B) * H * ((S_q + 2 * kBM - 1) / (2 * kBM)) * n_split;
+  if (n_units > INT_MAX) return VIDATTN_ERR_BAD_SHAPE;
+  const int sms = device_sms(dev);
+  const bool persist =
+      n_split == 1 && use_persistent(n_units, sms, (S_kv + kBN - 1) / kBN, D);
+  *grid_ctas = launch_grid(n_units, sms, persist);
+  *key_splits = n_split;
+  *persistent = persist ? 1 : 0;
+  return VIDATTN_OK;
 }
 
 VIDATTN_API int vidattn_kernels_per_call(const int32_t* seg_q, const int32_t* seg_kv, int B,
