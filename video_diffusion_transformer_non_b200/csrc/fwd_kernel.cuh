@@ -14,19 +14,24 @@
 // skipped, not masked (same paper, Appendix A, Table 4, group 2, row
 // "HunyuanVideo-1.5: RESOURCE_EXHAUSTED at 720p").
 //
-// One CTA = (b, h, 256 query rows as two 128-row tiles Q0, Q1).  384 threads:
-//   warps 0-3  softmax for Q0 (TMEM lanes 0-127 = the tile's rows)
-//   warps 4-7  softmax for Q1
+// Work unit = (b, h, 256 query rows as two 128-row tiles Q0, Q1[, one of
+// n_split ranges of the key tiles]).  One CTA per unit, or a persistent grid
+// of one CTA per SM, each CTA looping over units with every barrier phase
+// running on.  384 threads:
+//   warps 0-3  softmax for Q0 (TMEM lanes 0-127 = the tile's rows), epilogue
+//   warps 4-7  softmax for Q1, epilogue
 //   warp  8    allocates TMEM; runs the tensor-core schedule converged, an
 //              elected lane issuing every tcgen05.mma and commit
 //   warp  9    runs the load schedule converged, an elected lane issuing
-//              every TMA load (Q0, Q1 once; then K_j, V_j)
-//   warps 10-11 idle
+//              every TMA load (Q0, Q1 once per unit; then K_j, V_j)
+//   warp  10   with ids or windows: lists each unit's visited key tiles
+//   warp  11   idle
 // Tensor memory (512 columns x 128 lanes, fp32), D = 128:
 //   [0,128) S0 / P0   [128,256) S1 / P1   [256,384) O0   [384,512) O1
 // P (bf16, two per column) overwrites the first 64 columns of its S tile.
 // D = 64 (kSepP): S0, S1 in [0,256), P0, P1 in [256,384), O0, O1 in [384,512);
-// the softmax moves its S row into registers and releases S at once.
+// the softmax moves its S row into registers and releases S once P is
+// computed (the exponentials consume the S registers as they go).
 // Shared memory: Q0, Q1, then a ring of kStages K-or-V tiles; every tile is
 // [D/64][128 rows][64 columns] bf16 written by TMA with 128-byte swizzle.
 //
