@@ -50,14 +50,20 @@ __global__ void __launch_bounds__(128) seg_tile_classify_kernel(
 
 // 3D neighbourhood windows (vidattn_fwd_window): for every (b, 128-token
 // tile) of coord_q and coord_kv, the bounding box of the tile's (t, h, w)
-// coordinates, int4 {t_lo | t_hi << 16, h_lo | h_hi << 16, w_lo | w_hi << 16, 0}
-// (coordinates packed per token as t << 22 | h << 11 | w).  The attention
-// kernel skips a key tile whose box misses the union of its queries' windows
-// and takes the unmasked path where the box lies inside every query's window.
-// Launch shape as seg_tile_classify_kernel.
+// coordinates, int4 {t_lo | t_hi << 16, h_lo | h_hi << 16, w_lo | w_hi << 16,
+// raster} (coordinates packed per token as t << 22 | h << 11 | w).  The
+// attention kernel skips a key tile whose box misses the union of its
+// queries' windows and takes the unmasked path where the box lies inside
+// every query's window.  raster = 1 when every token x of the tile sits at
+// the raster position of its index in a volume of rows of Wg tokens (t = x /
+// (Hg Wg), h = x / Wg mod Hg, w = x mod Wg) and Wg >= kRasterMinW: the
+// kernel then builds a row's mask from the tile index alone.  Launch shape
+// as seg_tile_classify_kernel.
+constexpr int kRasterMinW = 10;   // at most 16 (t, h) rows in a 128-key tile
 __global__ void __launch_bounds__(128) win_tile_bbox_kernel(
     const int32_t* __restrict__ coord_q, const int32_t* __restrict__ coord_kv,
-    int4* __restrict__ q_box, int4* __restrict__ kv_box, int S_q, int S_kv) {
+    int4* __restrict__ q_box, int4* __restrict__ kv_box, int S_q, int S_kv, int T, int Hg,
+    int Wg) {
   const int which = blockIdx.z;
   const int b = blockIdx.y;
   const int tile = blockIdx.x;
@@ -67,12 +73,17 @@ __global__ void __launch_bounds__(128) win_tile_bbox_kernel(
   const int32_t* coord = (which ? coord_kv : coord_q) + static_cast<int64_t>(b) * S;
   const int idx = tile * kSegTile + threadIdx.x;
   int lo[3] = {INT_MAX, INT_MAX, INT_MAX}, hi[3] = {INT_MIN, INT_MIN, INT_MIN};
+  bool raster = Wg >= kRasterMinW;
   if (idx < S) {
     const uint32_t c = static_cast<uint32_t>(__ldg(coord + idx));
     lo[0] = hi[0] = int(c >> 22);
     lo[1] = hi[1] = int((c >> 11) & 2047u);
     lo[2] = hi[2] = int(c & 2047u);
+    const int row = idx / Wg;
+    raster = raster && row / Hg < T &&
+             c == (uint32_t(row / Hg) << 22 | uint32_t(row % Hg) << 11 | uint32_t(idx % Wg));
   }
+  raster = __syncthreads_and(raster) != 0;
 #pragma unroll
   for (int a = 0; a < 3; ++a) {
 #pragma unroll
@@ -100,7 +111,7 @@ __global__ void __launch_bounds__(128) win_tile_bbox_kernel(
       packed[a] = l | (h << 16);
     }
     int4* dst = (which ? kv_box : q_box) + static_cast<int64_t>(b) * n_tiles + tile;
-    *dst = make_int4(packed[0], packed[1], packed[2], 0);
+    *dst = make_int4(packed[0], packed[1], packed[2], raster ? 1 : 0);
   }
 }
 

@@ -69,6 +69,11 @@ constexpr int kMaxListedTiles = 2048;
 // Threads that read a unit's tile list (loader warp, MMA warp, softmax
 // warpgroups); each arrives once when it is done with the list.
 constexpr int kListReaders = 320;
+// A list entry: the key tile's index | kListRaster when its keys lie in raster
+// order (windows; see win_tile_bbox_kernel) | bit 30 + i when Q tile i needs
+// the mask on it.
+constexpr int kListTileMask = 0x1FFFFFFF;
+constexpr int kListRaster = 1 << 29;
 
 struct FwdParams {
   const int32_t* seg_q;     // [B,S_q] or null
@@ -376,6 +381,35 @@ __device__ __noinline__ uint4 tile_mask_call(const int32_t* kinfo, int mode, int
   return tile_mask(kinfo, mode, my_seg, ws0, ws1, ws2, k0, k1, k2, n_lim);
 }
 
+// Window variant: the mask of one query row (window starts ws0..2, sizes
+// k0..2) over key tile j whose keys lie in raster order in a volume of rows
+// of Wg tokens and Hg rows per frame: key x of the tile is token j*128 + x at
+// (t, h, w) = its raster position, so the tile's keys are the runs of the
+// (t, h) rows it crosses, and a row sees the keys of a run whose (t, h) is in
+// its window, w in [ws2, ws2 + k2).  Keys at or past n_lim are hidden.  The
+// same bits as tile_mask's in mode 2, from the tile index alone.
+__device__ __forceinline__ uint4 raster_mask(int j, int n_lim, int Hg, int Wg, int ws0, int ws1,
+                                            int ws2, int k0, int k1, int k2) {
+  const int k_first = j * kBN;
+  const int r0 = k_first / Wg;                 // (t, h) row of the tile's first key
+  int xa = r0 * Wg - k_first;                  // tile offset of that row's w = 0 (<= 0)
+  int t = r0 / Hg, h = r0 - (r0 / Hg) * Hg;
+  const int wlo = max(ws2, 0), whi = min(ws2 + k2, Wg);
+  uint32_t mb[4] = {0u, 0u, 0u, 0u};
+  for (; xa < n_lim; xa += Wg) {
+    if (uint32_t(t - ws0) < uint32_t(k0) && uint32_t(h - ws1) < uint32_t(k1)) {
+      const int lo = max(xa + wlo, 0);
+      const int hi = min(xa + whi, n_lim);
+      if (lo < hi) set_bit_range(mb, lo, hi);
+    }
+    if (++h == Hg) {
+      h = 0;
+      ++t;
+    }
+  }
+  return make_uint4(mb[0], mb[1], mb[2], mb[3]);
+}
+
 // One thread's row of a 128-column S tile from tensor memory.
 __device__ __forceinline__ void load_s_row(uint32_t taddr, float (&s)[kBN]) {
   uint32_t sr[4][32];
@@ -564,7 +598,7 @@ struct UnitSched {
   // n_kv once the unit's range is done
   __device__ __forceinline__ int tile(int t, int prev_j) const {
     if (t >= t1) return n_kv;
-    if (list != nullptr) return list[t] & 0x3FFFFFFF;
+    if (list != nullptr) return list[t] & kListTileMask;
     return walk.next(prev_j + 1);
   }
 };
@@ -996,7 +1030,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             m0 = last_ragged || !(q0.z && ks.z && q0.x == ks.x) || causal_partial(p, x.pair, 0, jj);
             m1 = last_ragged || !(q1.z && ks.z && q1.x == ks.x) || causal_partial(p, x.pair, 1, jj);
           }
-          entry = jj | (m0 ? (1 << 30) : 0) | (m1 ? int(1u << 31) : 0);
+          entry = jj | (m0 ? (1 << 30) : 0) | (m1 ? int(1u << 31) : 0) |
+                  ((has_win && ks.w == 1) ? kListRaster : 0);
         }
         const unsigned ballot = __ballot_sync(0xffffffffu, act);
         if (act) list[cnt + __popc(ballot & ((1u << lane) - 1u))] = entry;
@@ -1045,6 +1080,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int4 my_qs;
       make_walk(p, x.b, pair, qi, &my_qs);
       const UnitSched sched = unit_sched(p, x, list, n_list);
+      // window variant: the row's window starts, once per unit (masks of
+      // key tiles in raster order are built from them and the tile index)
+      int ws0 = 0, ws1 = 0, ws2 = 0;
+      if (kMaskFast && has_win) {
+        const uint32_t qc =
+            row_valid ? uint32_t(__ldg(p.coord_q + static_cast<int64_t>(x.b) * p.S_q + row)) : 0u;
+        const WinRow wr = win_row(p, qc);
+        ws0 = wr.s[0];
+        ws1 = wr.s[1];
+        ws2 = wr.s[2];
+      }
 
       float m_run = -INFINITY;   // running max of scale*log2(e)*s, the offset of P
       float l_run = 0.f;         // running sum of P (fp32, before bf16 rounding)
@@ -1052,8 +1098,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int t = sched.t0;
       for (int j = sched.tile(t, t - 1); j < sched.n_kv; ++t, ++lt, ++T, j = sched.tile(t, j)) {
         bool masked;
+        bool raster = false;   // window variant: a key tile in raster order
         if (list != nullptr) {
           masked = (list[t] >> (30 + qi)) & 1;
+          raster = kMaskFast && (list[t] & kListRaster) != 0;
         } else {
           masked = (ragged_kv && j == p.n_kv_tiles - 1) || causal_partial(p, pair, qi, j) || has_win;
           if (has_seg) {
@@ -1066,7 +1114,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // for S, so their latency hides behind it (warp-uniform: masked is the
         // same for every row of a Q tile).
         int32_t pre[4] = {0, 0, 0, 0};
-        if (masked && has_sum) {
+        if (masked && has_sum && !raster) {
           // the keys' ids or coordinates (tile summaries come with one or the other)
           const int32_t* src = (has_win ? p.coord_kv : p.seg_kv) + static_cast<int64_t>(x.b) * p.S_kv;
 #pragma unroll
@@ -1104,13 +1152,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // it with the tensor core's Q K^T (measured +3 % on a 480p windowed
         // call) instead of putting it on the chain after S; the slot is
         // free, as the previous masked tile's mask was built before its
-        // __syncwarp.  The exact paths reread the same slot.
+        // __syncwarp.  A key tile in raster order needs no slot: its mask
+        // comes from the tile index.  The exact paths use this mask.
         uint32_t mb_early[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
         bool have_mask = false;
         if (kMaskFast && masked && has_sum) {
+          if (raster) {
+            const int j0 = j * kBN;
+            const int n_valid = min(kBN, p.S_kv - j0);
+            const int n_lim =
+                p.causal ? max(0, min(n_valid, row + p.causal_off - j0 + 1)) : n_valid;
+            const uint4 mk = raster_mask(j, n_lim, p.win_extent[1], p.win_extent[2], ws0, ws1, ws2,
+                                         p.win_size[0], p.win_size[1], p.win_size[2]);
+            mb_early[0] = mk.x;
+            mb_early[1] = mk.y;
+            mb_early[2] = mk.z;
+            mb_early[3] = mk.w;
+          } else {
 #pragma unroll
-          for (int m = 0; m < 4; ++m) kinfo[lane + 32 * m] = pre[m];
-          build_mask(mb_early);
+            for (int m = 0; m < 4; ++m) kinfo[lane + 32 * m] = pre[m];
+            build_mask(mb_early);
+          }
           have_mask = true;
         }
         VIDATTN_TR(1 + qi, T, 0);
@@ -1145,8 +1207,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           if (exact) {
             // the mask first: no S register is live across its call
-            uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
-            if (masked) build_mask(mb);
+            uint32_t mb[4] = {mb_early[0], mb_early[1], mb_early[2], mb_early[3]};
+            if (masked && !have_mask) build_mask(mb);
             load_s_row(tS, s);
             float tile_max;
             if (!slow) {
@@ -1268,8 +1330,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // tensor memory (S is intact: no P has been written yet).  The sum
             // restarts: a failed running-offset attempt leaves its sum in rs.
             rs = 0.f;
-            uint32_t mb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
-            if (masked) build_mask(mb);
+            uint32_t mb[4] = {mb_early[0], mb_early[1], mb_early[2], mb_early[3]};
+            if (masked && !have_mask) build_mask(mb);
             // this chunk's 32 mask bits (kk is a runtime index: select, don't index)
             auto chunk_bits = [&](int kk) {
               return kk == 0 ? mb[0] : (kk == 1 ? mb[1] : (kk == 2 ? mb[2] : mb[3]));

@@ -673,7 +673,8 @@ VIDATTN_API int vidattn_fwd_window(const void* q, const void* k, const void* v,
   int4* q_box = reinterpret_cast<int4*>(buf);
   int4* kv_box = q_box + size_t(B) * nq;
   dim3 grid(nq > nk ? nq : nk, B, 2);
-  win_tile_bbox_kernel<<<grid, 128, 0, stream>>>(coord_q, coord_kv, q_box, kv_box, S_q, S_kv);
+  win_tile_bbox_kernel<<<grid, 128, 0, stream>>>(coord_q, coord_kv, q_box, kv_box, S_q, S_kv,
+                                                  T, Hg, Wg);
   if (cudaGetLastError() != cudaSuccess) return VIDATTN_ERR_CUDA;
   WinSpec win{coord_q, coord_kv, {win_t, win_h, win_w}, {T, Hg, Wg},
               (flags & VIDATTN_WINDOW_CLAMPED) ? 1 : 0};
