@@ -87,6 +87,7 @@ struct FwdParams {
   const int32_t* coord_q;   // [B,S_q]
   const int32_t* coord_kv;  // [B,S_kv]
   int win_size[3], win_extent[3], win_clamped;
+  FastDiv div_wg, div_hg;   // by win_extent[2] (Wg) and win_extent[1] (Hg)
   uint16_t* out;            // bf16 [B,H,S_q,D]
   float* lse;               // fp32 [B,H,S_q]
   int* err;                 // device error word (bit kErrTimeout: a wait timed out)
@@ -388,12 +389,15 @@ __device__ __noinline__ uint4 tile_mask_call(const int32_t* kinfo, int mode, int
 // (t, h) rows it crosses, and a row sees the keys of a run whose (t, h) is in
 // its window, w in [ws2, ws2 + k2).  Keys at or past n_lim are hidden.  The
 // same bits as tile_mask's in mode 2, from the tile index alone.
-__device__ __forceinline__ uint4 raster_mask(int j, int n_lim, int Hg, int Wg, int ws0, int ws1,
-                                            int ws2, int k0, int k1, int k2) {
+__device__ __forceinline__ uint4 raster_mask(const FwdParams& p, int j, int n_lim, int ws0,
+                                            int ws1, int ws2) {
+  const int Hg = p.win_extent[1], Wg = p.win_extent[2];
+  const int k0 = p.win_size[0], k1 = p.win_size[1], k2 = p.win_size[2];
   const int k_first = j * kBN;
-  const int r0 = k_first / Wg;                 // (t, h) row of the tile's first key
+  const int r0 = int(fastdiv(uint32_t(k_first), p.div_wg));   // (t, h) row of the first key
   int xa = r0 * Wg - k_first;                  // tile offset of that row's w = 0 (<= 0)
-  int t = r0 / Hg, h = r0 - (r0 / Hg) * Hg;
+  int t = int(fastdiv(uint32_t(r0), p.div_hg));
+  int h = r0 - t * Hg;
   const int wlo = max(ws2, 0), whi = min(ws2 + k2, Wg);
   uint32_t mb[4] = {0u, 0u, 0u, 0u};
   for (; xa < n_lim; xa += Wg) {
@@ -1162,8 +1166,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const int n_valid = min(kBN, p.S_kv - j0);
             const int n_lim =
                 p.causal ? max(0, min(n_valid, row + p.causal_off - j0 + 1)) : n_valid;
-            const uint4 mk = raster_mask(j, n_lim, p.win_extent[1], p.win_extent[2], ws0, ws1, ws2,
-                                         p.win_size[0], p.win_size[1], p.win_size[2]);
+            const uint4 mk = raster_mask(p, j, n_lim, ws0, ws1, ws2);
             mb_early[0] = mk.x;
             mb_early[1] = mk.y;
             mb_early[2] = mk.z;

@@ -1,6 +1,7 @@
 // Hand-written PTX wrappers for sm_100a: mbarriers, TMA tensor loads,
 // tcgen05 (TMEM allocation, MMA with TMEM accumulators, TMEM loads/stores)
-// and the exp2 unit.  Used only by the attention kernels in this directory.
+// and the exp2 unit, and division by a run-time invariant.  Used only by the
+// kernels in this directory.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -288,6 +289,22 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   r.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
   r.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
   return r;
+}
+
+// n / d for 0 <= n < 2^31 by one multiply-high, add and shift (Granlund and
+// Montgomery, "Division by invariant integers using multiplication", 1994,
+// the round-up multiplier: l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1).
+struct FastDiv {
+  uint32_t d, m, l;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((uint64_t(1) << l) < d) ++l;
+  const uint64_t m = ((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1;
+  return FastDiv{d, uint32_t(m), l};
+}
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.m) + n) >> f.l;
 }
 
 }  // namespace vidattn

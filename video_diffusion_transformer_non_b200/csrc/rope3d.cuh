@@ -32,22 +32,6 @@ constexpr int kRopeThreads = 256;
 constexpr int kRopeTokens = 8;
 constexpr int kRopeMaxD = 128;
 
-// n / d for 0 <= n < 2^31 by one multiply-high, add and shift (Granlund and
-// Montgomery, "Division by invariant integers using multiplication", 1994,
-// the round-up multiplier: l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1).
-struct FastDiv {
-  uint32_t d, m, l;
-};
-inline FastDiv make_fastdiv(uint32_t d) {
-  uint32_t l = 0;
-  while ((uint64_t(1) << l) < d) ++l;
-  const uint64_t m = ((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1;
-  return FastDiv{d, uint32_t(m), l};
-}
-__device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDiv& f) {
-  return (__umulhi(n, f.m) + n) >> f.l;
-}
-
 struct RopeParams {
   const uint16_t* in[2];
   uint16_t* out[2];

@@ -413,6 +413,8 @@ int launch_fwd(int dev, const void* q, const void* k, const void* v, const int32
       p.win_extent[a] = win->extent[a];
     }
     p.win_clamped = win->clamped;
+    p.div_wg = make_fastdiv(uint32_t(win->extent[2]));
+    p.div_hg = make_fastdiv(uint32_t(win->extent[1]));
   }
   p.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
 #ifdef VIDATTN_TRACE
