@@ -399,19 +399,24 @@ __device__ __forceinline__ uint4 raster_mask(const FwdParams& p, int j, int n_li
   int t = int(fastdiv(uint32_t(r0), p.div_hg));
   int h = r0 - t * Hg;
   const int wlo = max(ws2, 0), whi = min(ws2 + k2, Wg);
-  uint32_t mb[4] = {0u, 0u, 0u, 0u};
+  // the mask as two 64-bit halves: bits [a, e) of a half, 0 <= a < e <= 64,
+  // are (~0 >> (64 - (e - a))) << a
+  uint64_t m01 = 0, m23 = 0;
   for (; xa < n_lim; xa += Wg) {
     if (uint32_t(t - ws0) < uint32_t(k0) && uint32_t(h - ws1) < uint32_t(k1)) {
       const int lo = max(xa + wlo, 0);
       const int hi = min(xa + whi, n_lim);
-      if (lo < hi) set_bit_range(mb, lo, hi);
+      const int a0 = min(lo, 64), e0 = min(hi, 64);
+      const int a1 = max(lo, 64) - 64, e1 = max(hi, 64) - 64;
+      if (a0 < e0) m01 |= (~0ull >> (64 - (e0 - a0))) << a0;
+      if (a1 < e1) m23 |= (~0ull >> (64 - (e1 - a1))) << a1;
     }
     if (++h == Hg) {
       h = 0;
       ++t;
     }
   }
-  return make_uint4(mb[0], mb[1], mb[2], mb[3]);
+  return make_uint4(uint32_t(m01), uint32_t(m01 >> 32), uint32_t(m23), uint32_t(m23 >> 32));
 }
 
 // One thread's row of a 128-column S tile from tensor memory.
