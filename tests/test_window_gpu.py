@@ -122,6 +122,21 @@ def test_shuffled_token_order_and_per_sample_coordinates():
     check_window(c, win, "shuffled sample 1")
 
 
+def test_raster_and_staged_key_tiles_in_one_call():
+    """Keys in raster order except two swapped tokens in the third key tile:
+    that tile takes the staged-coordinate mask, the others the raster-order
+    mask from the tile index; one call, B = 2 with only sample 0 altered, so
+    the two samples' tiles differ too."""
+    grid = (3, 12, 24)
+    S = int(np.prod(grid))
+    c = wl.make_random(2, 2, S, S, 128, 31)
+    ck = wl.raster_coords(grid, 2).copy()
+    ck[0, [2 * 128 + 5, 2 * 128 + 77]] = ck[0, [2 * 128 + 77, 2 * 128 + 5]]
+    cq = wl.raster_coords(grid, 2)
+    win = dict(coord_q=cq, coord_kv=ck, size=(3, 5, 7), extent=grid, clamped=True)
+    check_window(c, win, "raster with one staged tile")
+
+
 def test_queries_and_keys_from_different_token_sets():
     """S_q != S_kv: queries are one frame, keys the whole volume."""
     grid = (5, 8, 16)
