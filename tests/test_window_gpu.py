@@ -137,6 +137,19 @@ def test_raster_and_staged_key_tiles_in_one_call():
     check_window(c, win, "raster with one staged tile")
 
 
+def test_keys_a_raster_prefix_of_the_volume():
+    """Keys are the first 500 tokens of the volume in raster order (a ragged
+    last key tile, a last (t, h) row cut short), queries the whole volume:
+    raster-order masks end at the sequence, and queries whose window holds
+    no key get out = 0, lse = -inf."""
+    grid = (3, 12, 24)
+    ck_full = wl.raster_coords(grid, 1)
+    ck = np.ascontiguousarray(ck_full[:, :500])
+    c = wl.make_random(1, 2, ck_full.shape[1], 500, 128, 33)
+    win = dict(coord_q=ck_full, coord_kv=ck, size=(1, 3, 5), extent=grid, clamped=False)
+    check_window(c, win, "raster prefix keys")
+
+
 def test_queries_and_keys_from_different_token_sets():
     """S_q != S_kv: queries are one frame, keys the whole volume."""
     grid = (5, 8, 16)
