@@ -179,7 +179,12 @@ VIDATTN_API int vidattn_fwd_ex(const void* q, const void* k, const void* v,
  *   the rest              as vidattn_fwd.
  *
  * Key tiles (128 keys) whose coordinate box misses every window of a CTA's
- * 256 queries are never loaded; tiles inside every window skip the mask.  Two
+ * 256 queries are never loaded; tiles inside every window skip the mask.  At
+ * D = 128 the mask of a key tile whose tokens all sit at the raster position
+ * of their index (token x at t = x / (Hg Wg), h = x / Wg mod Hg, w = x mod
+ * Wg) with Wg >= 10 is built from the tile index alone, which is faster than
+ * the general path (keys' coordinates staged in shared memory); results are
+ * the same either way.  Two
  * kernels per call (tile boxes, then the attention); the tile boxes use the
  * scratch of vidattn_fwd (per device and stream).  Errors: NULL coordinates
  * return VIDATTN_ERR_NULL; bad window sizes, extents, S_kv or flag bits
